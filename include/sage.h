@@ -1,0 +1,183 @@
+/*
+ * sage.h -- C ABI of libsage.so: SageAttention-style quantized attention
+ * forward for NVIDIA B200 (sm_100a).
+ *
+ * Method sources (web pages):
+ *   [SA1]   "SageAttention: Accurate 8-Bit Attention for Plug-and-Play
+ *           Inference Acceleration" (review page): Algorithm 1 (SAGEAttn-B),
+ *           Eq. 4-5, Eq. 6 (Smooth K), implementation details 1-2.
+ *   [SA2++] "SageAttention2++: A More Efficient Implementation of
+ *           SageAttention2" (review page): section "核心公式" (delta_Q,
+ *           delta_K, delta_P, delta_V formulas; Eq. (1)-(2)).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are dense, row-major, in device memory unless the name says
+ *     "host".  Q and O are [B, H, N, d]; K and V are [B, H_kv, N, d]
+ *     (the (B, H, N, d) shapes of [SA1] Table 7).  d is the innermost axis.
+ *   - d must be 64 or 128; H must be a multiple of H_kv (query head h reads
+ *     kv head h / (H / H_kv)).  N may be any value >= 0; the last 128-token
+ *     block of a ragged sequence is short.  B == 0 or N == 0 is a no-op.
+ *   - q, k, v, o, q_hat, k_hat, v_hat must be 16-byte aligned (TMA and
+ *     vector access); fp32 arrays 4-byte aligned.  Violations return
+ *     SAGE_ERR_MISALIGNED before anything is launched.
+ *   - The caller owns all memory.  Calls keep no state between them.
+ *   - `stream` is a cudaStream_t passed as an opaque pointer (NULL = the
+ *     legacy default stream).  Calls are stream-ordered and asynchronous:
+ *     the returned status covers argument checks and launch errors only.
+ *     Execution errors surface at the caller's next synchronization, or
+ *     through sage_get_device_error().
+ *   - Inputs holding NaN or Inf are outside the contract.
+ *   - There is no CPU or other-architecture fallback: a current device
+ *     that is not compute capability 10.0 gives SAGE_ERR_DEVICE.
+ *   - Quantization blocks are 128 tokens of one head (b_q = b_kv = 128),
+ *     so the scale arrays have nb = ceil(N / 128) entries per head.
+ */
+#ifndef SAGE_H_
+#define SAGE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SAGE_OK = 0,
+  SAGE_ERR_INVALID_ARG = 1,     /* null pointer, negative size, sm_scale <= 0 or not finite */
+  SAGE_ERR_UNSUPPORTED = 2,     /* d not in {64,128}, H % H_kv != 0, unknown variant        */
+  SAGE_ERR_MISALIGNED = 3,      /* a device pointer not 16-byte aligned                      */
+  SAGE_ERR_DEVICE = 4,          /* current device is not compute capability 10.0 (B200)      */
+  SAGE_ERR_CUDA = 5,            /* a CUDA runtime / driver call failed                       */
+  SAGE_ERR_DEVICE_TIMEOUT = 6,  /* a kernel gave up on a bounded wait (see device error)     */
+  SAGE_ERR_NO_MEMORY = 7        /* stream-ordered allocation failed / workspace too small    */
+} sage_status_t;
+
+typedef enum {
+  /* INT8 Q K^T, P~ and V in fp16 for P~V, fp32 accumulator ([SA1] Algorithm 1). */
+  SAGE_VARIANT_B = 0,
+  /* INT8 Q K^T, P~ and V in FP8 E4M3 ("8+8" of [SA2++]): static delta_P = 1/448,
+   * per-channel delta_V = colmax|V| / 448, fp32 accumulator. */
+  SAGE_VARIANT_8P8 = 1
+} sage_variant_t;
+
+/*
+ * Pre-pass for Q and K ([SA1] Algorithm 1 steps 1-2, Eq. 6; [SA2++] delta_Q,
+ * delta_K formulas).
+ *   q      : fp16 [B,H,N,d]        k : fp16 [B,H_kv,N,d]       (inputs)
+ *   q_hat  : int8 [B,H,N,d]        = RNE(x_q / delta_q[blk]), x_q = fp32(q) * sm_scale
+ *   k_hat  : int8 [B,H_kv,N,d]     = RNE(x_k / delta_k[blk]), x_k = fp32(k) - mean_k[c]
+ *   delta_q: fp32 [B,H,nb]         = max|x_q over the block| / 127  (0 for an all-zero block)
+ *   delta_k: fp32 [B,H_kv,nb]      = max|x_k over the block| / 127
+ *   mean_k : fp32 [B,H_kv,d]       = (1/N) sum_t k[t,c]; the sum is exact (fixed point,
+ *                                    units of 2^-24), converted to fp64, divided by N
+ *                                    in fp64, rounded once to fp32.
+ * Both divisions are IEEE fp32 round-to-nearest; codes lie in [-127, 127].
+ * Results are bit-identical whatever the launch configuration.
+ * Scratch: takes ceil(N/256)*B*H_kv*d*8 bytes of stream-ordered device memory
+ * (cudaMallocAsync on `stream`, freed on `stream`).
+ */
+sage_status_t sage_smooth_quant_qk(const void* q, const void* k, int B, int H, int H_kv,
+                                   int N, int d, float sm_scale, int8_t* q_hat, int8_t* k_hat,
+                                   float* delta_q, float* delta_k, float* mean_k, void* stream);
+
+/*
+ * FP8 E4M3 quantization of V for the 8+8 variant ([SA2++] delta_V formula and
+ * Eq. (2) with a general V_r).
+ *   v      : fp16 [B,H_kv,N,d]
+ *   v_r    : top of the code range (448 for 8+8); must be in (0, 448]
+ *   v_hat  : uint8 E4M3 codes, [B,H_kv,N,d] (the layout of v; see sage_v_hat_layout)
+ *            = e4m3_rne_satfinite(fp32(v) / delta_v[c])
+ *   delta_v: fp32 [B,H_kv,d] = max_t |v[t,c]| / v_r (IEEE fp32 division; 0 -> codes 0)
+ * Scratch: ceil(N/256)*B*H_kv*d*4 bytes, stream-ordered as above.
+ */
+sage_status_t sage_quant_v_fp8(const void* v, int B, int H_kv, int N, int d, float v_r,
+                               uint8_t* v_hat, float* delta_v, void* stream);
+
+/*
+ * Attention on pre-quantized operands ([SA1] Algorithm 1 steps 3-9, Eq. 4-5):
+ * per 128-row q block and ascending 128-key kv tiles,
+ *   S = int32(q_hat k_hat^T) * delta_q[i] * delta_k[j]   (tcgen05 kind::i8)
+ *   online softmax (running max m, row sum l, rescale of O)
+ *   O += P~ V  (variant B: fp16 P~ and fp16 V; 8+8: e4m3(448 P~) and v_hat)
+ *   O = O / l  (8+8: times delta_v[c] / 448), rounded to fp16.
+ *   v_or_vhat: fp16 V for SAGE_VARIANT_B, E4M3 codes for SAGE_VARIANT_8P8
+ *   delta_v  : fp32 [B,H_kv,d] for 8+8, ignored (may be NULL) for B
+ *   o        : fp16 [B,H,N,d] output
+ *   causal   : 0 or 1; square, top-left aligned mask (key t visible to query r iff t <= r)
+ * No scratch memory.
+ */
+sage_status_t sage_attn_fwd_quantized(const int8_t* q_hat, const int8_t* k_hat,
+                                      const float* delta_q, const float* delta_k,
+                                      const void* v_or_vhat, const float* delta_v, void* o,
+                                      int B, int H, int H_kv, int N, int d, int causal,
+                                      int variant, void* stream);
+
+/* Bytes of workspace sage_attn_fwd_ws needs for these sizes (0 for empty inputs). */
+size_t sage_attn_workspace_bytes(int B, int H, int H_kv, int N, int d, int variant);
+
+/*
+ * Whole forward pass ([SA1] Algorithm 1 with Smooth K; variant selects B or 8+8):
+ * pre-pass kernels then the attention kernel, on `stream`.
+ *   q, k, v : fp16 inputs as above; o : fp16 [B,H,N,d] output
+ *   sm_scale: softmax scale folded into the quantization of Q (> 0, finite;
+ *             1/sqrt(d) is the usual value)
+ * Intermediates (q_hat, k_hat, scales, mean_k, v_hat, scratch) come from
+ * cudaMallocAsync on `stream` and are freed on `stream` (_ws: from the
+ * caller's workspace of at least sage_attn_workspace_bytes() bytes,
+ * 256-byte aligned; SAGE_ERR_NO_MEMORY if it is smaller).
+ */
+sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H,
+                            int H_kv, int N, int d, int causal, float sm_scale, int variant,
+                            void* stream);
+sage_status_t sage_attn_fwd_ws(const void* q, const void* k, const void* v, void* o, int B,
+                               int H, int H_kv, int N, int d, int causal, float sm_scale,
+                               int variant, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * End-to-end call on HOST buffers: copies q, k, v (fp16, host memory; pinned
+ * memory gives full PCIe/C2C bandwidth) to the current device, runs
+ * sage_attn_fwd, copies o back to host memory and synchronizes `stream`
+ * before returning.  Device buffers are stream-ordered allocations freed
+ * before return.
+ */
+sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                                 void* o_host, int B, int H, int H_kv, int N, int d, int causal,
+                                 float sm_scale, int variant, void* stream);
+
+/* Layout of v_hat: 0 = [B,H_kv,N,d] (same as v).  Always 0 in this library. */
+int sage_v_hat_layout(void);
+
+/*
+ * Synchronizes `stream`, then reads and clears the library's device error
+ * word on the current device.  Returns SAGE_OK, SAGE_ERR_DEVICE_TIMEOUT if a
+ * kernel abandoned a bounded wait (it then skipped the rest of its work,
+ * released its tensor memory and exited), or SAGE_ERR_CUDA.
+ * If `detail` is not NULL it receives the raw error word (bit 0: timeout;
+ * bits 8-15: which wait gave up).
+ */
+sage_status_t sage_get_device_error(void* stream, uint32_t* detail);
+
+/* Upper bound, in nanoseconds, of every bounded wait inside the kernels
+ * (default 2e9).  Applies to launches made after the call; process-wide. */
+void sage_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * Failure-detection self-test: launches one CTA that waits on a shared-memory
+ * barrier nothing will ever complete, with the bound `timeout_ns`.  The wait
+ * gives up, records a timeout in the device error word and the kernel exits
+ * normally; sage_get_device_error() then reports SAGE_ERR_DEVICE_TIMEOUT.
+ */
+sage_status_t sage_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+
+/* Static description of a status code. */
+const char* sage_status_string(sage_status_t status);
+
+/* Library version, as "major.minor.patch". */
+const char* sage_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_H_ */

@@ -1,0 +1,249 @@
+"""Python binding of libsage.so: SageAttention-style quantized attention on B200.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/sage.h.  PyTorch supplies device
+memory and the current stream.  There is no fallback: if the library is not
+built, or the GPU is not a B200, the calls raise.
+
+Functions carry the names of the C entry points:
+  sage_smooth_quant_qk, sage_quant_v_fp8, sage_attn_fwd_quantized,
+  sage_attn_fwd, sage_attn_fwd_ws, sage_attn_workspace_bytes,
+  sage_attn_fwd_host, sage_get_device_error, sage_set_wait_timeout_ns,
+  sage_selftest_wait_timeout, sage_status_string, sage_version,
+  sage_v_hat_layout.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsage.so")
+
+SAGE_OK = 0
+SAGE_ERR_DEVICE_TIMEOUT = 6
+VARIANTS = {"B": 0, "8+8": 1}
+
+_c = ctypes
+_vp = _c.c_void_p
+_i = _c.c_int
+_f = _c.c_float
+
+_SIGS = {
+    "sage_smooth_quant_qk": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "sage_quant_v_fp8": (_i, [_vp, _i, _i, _i, _i, _f, _vp, _vp, _vp]),
+    "sage_attn_fwd_quantized": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "sage_attn_workspace_bytes": (_c.c_size_t, [_i, _i, _i, _i, _i, _i]),
+    "sage_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
+    "sage_attn_fwd_ws": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _c.c_size_t, _vp]),
+    "sage_attn_fwd_host": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
+    "sage_v_hat_layout": (_i, []),
+    "sage_get_device_error": (_i, [_vp, _c.POINTER(_c.c_uint32)]),
+    "sage_set_wait_timeout_ns": (None, [_c.c_uint64]),
+    "sage_selftest_wait_timeout": (_i, [_c.c_uint64, _vp]),
+    "sage_status_string": (_c.c_char_p, [_i]),
+    "sage_version": (_c.c_char_p, []),
+}
+
+_lib_handle = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libsage.so (raises if it has not been built)."""
+    global _lib_handle
+    if _lib_handle is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build the CUDA library first "
+                "(python -m quantized_attention_08_b200.build)")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib_handle = lib
+    return _lib_handle
+
+
+class SageError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {sage_status_string(status)} (status {status})")
+
+
+def sage_status_string(status: int) -> str:
+    return load_library().sage_status_string(int(status)).decode()
+
+
+def sage_version() -> str:
+    return load_library().sage_version().decode()
+
+
+def sage_v_hat_layout() -> int:
+    return load_library().sage_v_hat_layout()
+
+
+def _check(status: int, where: str):
+    if status != SAGE_OK:
+        raise SageError(status, where)
+
+
+def _stream(stream=None) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, dtype, name: str, cuda: bool = True):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if cuda and not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _variant(v) -> int:
+    return VARIANTS[v] if isinstance(v, str) else int(v)
+
+
+def _nb(N: int) -> int:
+    return (N + 127) // 128
+
+
+def sage_smooth_quant_qk(q: torch.Tensor, k: torch.Tensor, sm_scale: Optional[float] = None,
+                         out=None, stream=None):
+    """Smooth K, quantize Q*sm_scale and smoothed K per 128-token block.
+    Returns (q_hat int8, k_hat int8, delta_q fp32, delta_k fp32, mean_k fp32)."""
+    _need(q, torch.float16, "q")
+    _need(k, torch.float16, "k")
+    B, H, N, d = q.shape
+    Hk = k.shape[1]
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        dev = q.device
+        out = (torch.empty_like(q, dtype=torch.int8), torch.empty_like(k, dtype=torch.int8),
+               torch.empty(B, H, _nb(N), dtype=torch.float32, device=dev),
+               torch.empty(B, Hk, _nb(N), dtype=torch.float32, device=dev),
+               torch.empty(B, Hk, d, dtype=torch.float32, device=dev))
+    qh, kh, dq, dk, mk = out
+    st = load_library().sage_smooth_quant_qk(_ptr(q), _ptr(k), B, H, Hk, N, d, float(sm_scale),
+                                             _ptr(qh), _ptr(kh), _ptr(dq), _ptr(dk), _ptr(mk),
+                                             _stream(stream))
+    _check(st, "sage_smooth_quant_qk")
+    return out
+
+
+def sage_quant_v_fp8(v: torch.Tensor, v_r: float = 448.0, out=None, stream=None):
+    """E4M3 codes of V / delta_v with delta_v = colmax|V| / v_r per channel.
+    Returns (v_hat uint8 [B,Hkv,N,d], delta_v fp32 [B,Hkv,d])."""
+    _need(v, torch.float16, "v")
+    B, Hk, N, d = v.shape
+    if out is None:
+        out = (torch.empty_like(v, dtype=torch.uint8),
+               torch.empty(B, Hk, d, dtype=torch.float32, device=v.device))
+    vh, dv = out
+    st = load_library().sage_quant_v_fp8(_ptr(v), B, Hk, N, d, float(v_r), _ptr(vh), _ptr(dv),
+                                         _stream(stream))
+    _check(st, "sage_quant_v_fp8")
+    return out
+
+
+def sage_attn_fwd_quantized(q_hat, k_hat, delta_q, delta_k, v_or_vhat, delta_v=None, *,
+                            causal: bool = False, variant="B", o=None, stream=None):
+    """Attention on pre-quantized operands; returns o fp16 [B,H,N,d]."""
+    _need(q_hat, torch.int8, "q_hat")
+    _need(k_hat, torch.int8, "k_hat")
+    var = _variant(variant)
+    B, H, N, d = q_hat.shape
+    Hk = k_hat.shape[1]
+    if o is None:
+        o = torch.empty(B, H, N, d, dtype=torch.float16, device=q_hat.device)
+    st = load_library().sage_attn_fwd_quantized(
+        _ptr(q_hat), _ptr(k_hat), _ptr(delta_q), _ptr(delta_k), _ptr(v_or_vhat), _ptr(delta_v),
+        _ptr(o), B, H, Hk, N, d, int(bool(causal)), var, _stream(stream))
+    _check(st, "sage_attn_fwd_quantized")
+    return o
+
+
+def sage_attn_workspace_bytes(B: int, H: int, H_kv: int, N: int, d: int, variant="B") -> int:
+    return load_library().sage_attn_workspace_bytes(B, H, H_kv, N, d, _variant(variant))
+
+
+def sage_attn_fwd(q, k, v, *, causal: bool = False, sm_scale: Optional[float] = None,
+                  variant="B", o=None, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Whole SageAttention forward (Smooth K, quantize, attention); returns o fp16."""
+    _need(q, torch.float16, "q")
+    _need(k, torch.float16, "k")
+    _need(v, torch.float16, "v")
+    B, H, N, d = q.shape
+    Hk = k.shape[1]
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    lib = load_library()
+    if workspace is None:
+        st = lib.sage_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, Hk, N, d, int(bool(causal)),
+                               float(sm_scale), _variant(variant), _stream(stream))
+        _check(st, "sage_attn_fwd")
+    else:
+        st = lib.sage_attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, Hk, N, d,
+                                  int(bool(causal)), float(sm_scale), _variant(variant),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(stream))
+        _check(st, "sage_attn_fwd_ws")
+    return o
+
+
+def sage_attn_fwd_ws(q, k, v, workspace: torch.Tensor, *, causal: bool = False,
+                     sm_scale: Optional[float] = None, variant="B", o=None, stream=None):
+    """sage_attn_fwd with the intermediates carved from a caller workspace
+    (a CUDA tensor of at least sage_attn_workspace_bytes() bytes)."""
+    if workspace is None:
+        raise ValueError("workspace is required")
+    return sage_attn_fwd(q, k, v, causal=causal, sm_scale=sm_scale, variant=variant, o=o,
+                         workspace=workspace, stream=stream)
+
+
+def sage_attn_fwd_host(q_host, k_host, v_host, o_host, *, causal: bool = False,
+                       sm_scale: Optional[float] = None, variant="B", stream=None):
+    """End-to-end call on host (CPU, ideally pinned) fp16 tensors; o_host is written."""
+    for t, n in ((q_host, "q_host"), (k_host, "k_host"), (v_host, "v_host"), (o_host, "o_host")):
+        _need(t, torch.float16, n, cuda=False)
+        if t.is_cuda:
+            raise TypeError(f"{n} must be a host tensor")
+    B, H, N, d = q_host.shape
+    Hk = k_host.shape[1]
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    st = load_library().sage_attn_fwd_host(_ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(o_host),
+                                           B, H, Hk, N, d, int(bool(causal)), float(sm_scale),
+                                           _variant(variant), _stream(stream))
+    _check(st, "sage_attn_fwd_host")
+    return o_host
+
+
+def sage_get_device_error(stream=None):
+    """(status, raw error word); synchronizes the stream and clears the word."""
+    w = ctypes.c_uint32(0)
+    st = load_library().sage_get_device_error(_stream(stream), ctypes.byref(w))
+    return st, w.value
+
+
+def sage_set_wait_timeout_ns(ns: int):
+    load_library().sage_set_wait_timeout_ns(int(ns))
+
+
+def sage_selftest_wait_timeout(timeout_ns: int, stream=None):
+    _check(load_library().sage_selftest_wait_timeout(int(timeout_ns), _stream(stream)),
+           "sage_selftest_wait_timeout")

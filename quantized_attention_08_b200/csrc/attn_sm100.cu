@@ -1,0 +1,493 @@
+// attn_sm100.cu -- warp-specialised tcgen05 quantized attention for B200.
+//
+// [SA1] "SageAttention: Accurate 8-Bit Attention for Plug-and-Play Inference
+//       Acceleration", Algorithm 1 steps 3-9 and Eq. 4-5:
+//         S_i^j = INT8_Matmul(Q_i, K_j^T) * delta_Q[i] * delta_K[j]
+//         online softmax (m, l), O_i^j = rescale(O_i^{j-1}) + P~_i^j V_j
+//         O_i = diag(l_i)^-1 O_i
+// [SA2++] "SageAttention2++ ...", section "核心公式": the 8+8 P~V with
+//       static delta_P = 1/448 and per-channel delta_V.
+//
+// One CTA owns two 128-row q tiles of one (batch, head) and streams the kv
+// tiles of that head through a multi-stage TMA/mbarrier ring:
+//   warp 8      TMA producer (Q once, then K_j and V_j per stage)
+//   warp 9      MMA issuer: S_g = Q_g K_j^T (kind::i8 -> s32 in TMEM),
+//               O_g += P_g V_j (kind::f16 or kind::f8f6f4, P_g read from TMEM)
+//   warps 0-3   softmax of q tile 0, warps 4-7 softmax of q tile 1: each
+//               thread owns one row; it reads S from TMEM, keeps m and l in
+//               registers, writes P~ (fp16, or e4m3 of 448 P~) back into the
+//               TMEM columns of S, rescales its row of O when m moves, and
+//               finally normalises O and stores fp16.
+// Tensor memory (512 columns x 128 lanes): S_0 [0,128), S_1 [128,256),
+// O_0 [256,256+d), O_1 [384,384+d); P_g aliases the first columns of S_g.
+// Every wait is bounded (see mbar_wait); on expiry the CTA records the
+// error, abandons its work, drains its in-flight copies and MMAs, frees
+// tensor memory and exits.
+#include <cuda_fp16.h>
+#include <math.h>
+
+#include "sage_internal.h"
+
+namespace sage {
+
+constexpr int kBM = 128, kBN = 128;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kAttnThreads = 320;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLog2P448 = 8.807354922057604f;  // log2(448): P operand = 448 * P~
+
+template <int D, int VAR>
+struct Cfg {
+  static constexpr int NS = (VAR == 0 && D == 128) ? 3 : 4;  // ring stages
+  static constexpr int Q_BYTES = kBM * D;
+  static constexpr int K_BYTES = kBN * D;
+  static constexpr int V_BYTES = kBN * D * (VAR == 0 ? 2 : 1);
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * K_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NS * V_BYTES;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  // Q_hat / K_hat: K-major int8 rows of D bytes, swizzle span = row length.
+  static constexpr uint32_t QK_SW = (D == 128) ? SW_128B : SW_64B;
+  static constexpr uint32_t QK_SBO = 8 * D;
+  // V: MN-major (channels contiguous); fp16 V arrives as boxes of 64 channels.
+  static constexpr uint32_t V_ROW = (VAR == 0) ? 128 : D;  // bytes per kv row in a box
+  static constexpr uint32_t V_BOX_BYTES = kBN * V_ROW;
+  static constexpr uint32_t V_SW = (V_ROW == 128) ? SW_128B : SW_64B;
+  static constexpr uint32_t V_SBO = 8 * V_ROW;
+  static constexpr uint32_t V_LBO = V_BOX_BYTES;
+  static constexpr int PV_K = (VAR == 0) ? 16 : 32;  // kv rows per PV instruction
+  static constexpr uint32_t IDESC_QK = idesc(CF_S32, AF_S8, AF_S8, 0, 0, kBN, kBM);
+  static constexpr uint32_t IDESC_PV =
+      idesc(CF_F32, VAR == 0 ? AF_F16 : AF_E4M3, VAR == 0 ? AF_F16 : AF_E4M3, 0, 1, D, kBM);
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+struct AttnKParams {
+  const float* dq;  // [B*H, nqb]
+  const float* dk;  // [B*Hkv, nkvb]
+  const float* dv;  // [B*Hkv, D] (8+8)
+  __half* o;        // [B*H, N, D]
+  int H, Hkv, N, nqb, nkvb;
+  uint64_t timeout_ns;
+};
+
+// Bounded wait that ignores the abort flag: used to drain in-flight work.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > limit_ns) {
+      atomicOr(&g_error_word, ERR_TIMEOUT | (0xFFu << 8));
+      return;
+    }
+  }
+}
+
+// Softmax of one 128-column tile for this thread's row.  `a` holds the s32
+// scores on entry and the packed P operand on exit (fp16x2, or 4 x e4m3).
+// c = delta_q * delta_k * log2(e); m is the running max in the log2 domain.
+// Columns >= lim are masked (only when MASKED).  Returns the new max and
+// the row sum of this tile's (unrounded) P values.
+template <int VAR, bool MASKED>
+__device__ __forceinline__ float softmax_tile(uint32_t (&a)[128], float c, float m, int lim,
+                                              float& rowsum) {
+  if (MASKED) {
+#pragma unroll
+    for (int i = 0; i < 128; ++i)
+      if (i >= lim) a[i] = 0x80000000u;
+  }
+  int imax = static_cast<int>(a[0]);
+#pragma unroll
+  for (int i = 1; i < 128; ++i) imax = max(imax, static_cast<int>(a[i]));
+  // |imax| <= d * 127^2 < 2^22: the int -> float conversion is exact.
+  const float m_new = fmaxf(m, __fmul_rn(static_cast<float>(imax), c));
+  const float bias = (VAR == 1) ? (kLog2P448 - m_new) : -m_new;
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 128; i += 4) {
+    float p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      // exact int -> float: 1.5*2^23 + a has unit spacing for |a| < 2^22
+      const float f = __fsub_rn(__uint_as_float(a[i + e] + 0x4B400000u), 12582912.f);
+      p[e] = ex2_approx(__fmaf_rn(f, c, bias));
+      if (MASKED && i + e >= lim) p[e] = 0.f;
+    }
+    s0 += p[0] + p[1];
+    s1 += p[2] + p[3];
+    if (VAR == 0) {
+      a[i / 2] = pack_f16x2(p[0], p[1]);
+      a[i / 2 + 1] = pack_f16x2(p[2], p[3]);
+    } else {
+      a[i / 4] = pack_e4m3x2(p[0], p[1]) | (pack_e4m3x2(p[2], p[3]) << 16);
+    }
+  }
+  rowsum = s0 + s1;
+  return m_new;
+}
+
+template <int D, int VAR, bool CAUSAL>
+__global__ void __maxnreg__(200)
+    k_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+           const __grid_constant__ CUtensorMap tm_v, const AttnKParams p) {
+  using C = Cfg<D, VAR>;
+  constexpr int NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* bar_q = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + NS;
+  uint64_t* v_full = k_empty + NS;
+  uint64_t* v_empty = v_full + NS;
+  uint64_t* s_full = v_empty + NS;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* mma_done = pv_done + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int npairs = gridDim.x;
+  // causal: heaviest q-tile pairs first
+  const int pp = CAUSAL ? (npairs - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+  const int bh = blockIdx.y;
+  const int b = bh / p.H, h = bh % p.H;
+  const int zkv = b * p.Hkv + h / (p.H / p.Hkv);
+  const int qb0 = 2 * pp;
+  const bool has1 = qb0 + 1 < p.nqb;
+  const int nkv0 = CAUSAL ? min(qb0 + 1, p.nkvb) : p.nkvb;
+  const int nkv1 = CAUSAL ? min(qb0 + 2, p.nkvb) : p.nkvb;
+  const int nkv = has1 ? nkv1 : nkv0;
+  const uint64_t tlim = p.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&s_full[g], 1);
+      mbar_init(&p_full[g], 128);
+      mbar_init(&pv_done[g], 1);
+    }
+    mbar_init(mma_done, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * C::Q_BYTES);
+      tma_load_3d(&tm_q, bar_q, sQ, 0, qb0 * kBM, bh);
+      if (has1) tma_load_3d(&tm_q, bar_q, sQ + C::Q_BYTES, 0, (qb0 + 1) * kBM, bh);
+      int nk = 0, nv = 0;  // loads issued
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j % NS;
+        const uint32_t ph = ((j / NS) & 1) ^ 1;
+        if (!mbar_wait(&k_empty[s], ph, s_abort, tlim, 1)) break;
+        mbar_arrive_expect_tx(&k_full[s], C::K_BYTES);
+        tma_load_3d(&tm_k, &k_full[s], sK + s * C::K_BYTES, 0, j * kBN, zkv);
+        ++nk;
+        if (!mbar_wait(&v_empty[s], ph, s_abort, tlim, 2)) break;
+        mbar_arrive_expect_tx(&v_full[s], C::V_BYTES);
+        uint8_t* dst = sV + s * C::V_BYTES;
+        if (VAR == 0 && D == 128) {
+          tma_load_3d(&tm_v, &v_full[s], dst, 0, j * kBN, zkv);
+          tma_load_3d(&tm_v, &v_full[s], dst + C::V_BOX_BYTES, 64, j * kBN, zkv);
+        } else {
+          tma_load_3d(&tm_v, &v_full[s], dst, 0, j * kBN, zkv);
+        }
+        ++nv;
+      }
+      if (*s_abort) {  // let the copies still in flight land before the CTA exits
+        drain_wait(bar_q, 0, tlim);
+        for (int i = max(0, nk - NS); i < nk; ++i) drain_wait(&k_full[i % NS], (i / NS) & 1, tlim);
+        for (int i = max(0, nv - NS); i < nv; ++i) drain_wait(&v_full[i % NS], (i / NS) & 1, tlim);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+      bool ok = mbar_wait(bar_q, 0, s_abort, tlim, 3);
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int s = j % NS;
+        const uint32_t ph = (j / NS) & 1;
+        if (!mbar_wait(&k_full[s], ph, s_abort, tlim, 4)) break;
+        for (int g = 0; g < 2 && ok; ++g) {
+          if (g == 1 ? !has1 : (j >= nkv0)) continue;
+          // S_g (aliasing P_g) may be overwritten once PV_g(j-1) has read P_g
+          if (j > 0 && !mbar_wait(&pv_done[g], (j - 1) & 1, s_abort, tlim, 5)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk) {
+            const uint64_t ad = sdesc(aQ + g * C::Q_BYTES + kk * 32, 16, C::QK_SBO, C::QK_SW);
+            const uint64_t bd = sdesc(aK + s * C::K_BYTES + kk * 32, 16, C::QK_SBO, C::QK_SW);
+            mma_i8_ss(tmem + g * 128, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&s_full[g]);
+        }
+        if (!ok) break;
+        tc_commit(&k_empty[s]);
+        if (!mbar_wait(&v_full[s], ph, s_abort, tlim, 6)) break;
+        for (int g = 0; g < 2 && ok; ++g) {
+          if (g == 1 ? !has1 : (j >= nkv0)) continue;
+          if (!mbar_wait(&p_full[g], j & 1, s_abort, tlim, 7)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kBN / C::PV_K; ++kk) {
+            const uint64_t bd = sdesc(aV + s * C::V_BYTES + kk * C::PV_K * C::V_ROW, C::V_LBO,
+                                      C::V_SBO, C::V_SW);
+            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+            if (VAR == 0)
+              mma_f16_ts(tmem + 256 + g * 128, tmem + g * 128 + kk * 8, bd, C::IDESC_PV, acc);
+            else
+              mma_f8_ts(tmem + 256 + g * 128, tmem + g * 128 + kk * 8, bd, C::IDESC_PV, acc);
+          }
+          tc_commit(&pv_done[g]);
+        }
+        if (!ok) break;
+        tc_commit(&v_empty[s]);
+      }
+      tc_commit(mma_done);
+      drain_wait(mma_done, 0, tlim);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax
+    const int g = warp >> 2, wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const int qb = qb0 + g;
+    if (g == 0 || has1) {
+      const int nkv_g = g == 0 ? nkv0 : nkv1;
+      const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+      const uint32_t tS = tmem + lane_off + g * 128;
+      const uint32_t tO = tmem + lane_off + 256 + g * 128;
+      const float dq_l2e = __fmul_rn(p.dq[static_cast<size_t>(bh) * p.nqb + qb], kLog2e);
+      const float* dkp = p.dk + static_cast<size_t>(zkv) * p.nkvb;
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      float dk_next = dkp[0];
+      for (int j = 0; j < nkv_g; ++j) {
+        const float c = __fmul_rn(dq_l2e, dk_next);
+        if (j + 1 < nkv_g) dk_next = dkp[j + 1];
+        // tcgen05.ld/st below are warp-collective: every lane takes the same branch
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[g], j & 1, s_abort, tlim, 8))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t a[128];
+        SAGE_TMEM_LD32(tS + 0, a);
+        SAGE_TMEM_LD32(tS + 32, (a + 32));
+        SAGE_TMEM_LD32(tS + 64, (a + 64));
+        SAGE_TMEM_LD32(tS + 96, (a + 96));
+        tmem_wait_ld();
+        const int valid = p.N - j * kBN;  // keys left in this tile
+        const bool masked = (CAUSAL && j == qb) || valid < kBN;
+        float rs, m_new;
+        if (masked) {
+          const int lim = min(valid, (CAUSAL && j == qb) ? r + 1 : kBN);
+          m_new = softmax_tile<VAR, true>(a, c, m, lim, rs);
+        } else {
+          m_new = softmax_tile<VAR, false>(a, c, m, kBN, rs);
+        }
+        if (VAR == 0) {
+          SAGE_TMEM_ST32(tS + 0, a);
+          SAGE_TMEM_ST32(tS + 32, (a + 32));
+        } else {
+          SAGE_TMEM_ST32(tS + 0, a);
+        }
+        const float alpha = ex2_approx(m - m_new);  // 0 on the first tile
+        l = __fmaf_rn(alpha, l, rs);
+        if (j > 0 && __any_sync(0xFFFFFFFFu, m_new > m)) {
+          // O_g holds PV_g(j-1), complete: S_g(j) was issued after it.
+#pragma unroll 1
+          for (int cb = 0; cb < D / 32; ++cb) {
+            uint32_t o[32];
+            SAGE_TMEM_LD32(tO + cb * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            SAGE_TMEM_ST32(tO + cb * 32, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[g]);
+        m = m_new;
+      }
+      if (ok && __all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[g], (nkv_g - 1) & 1, s_abort, tlim, 9))) {
+        tc_fence_after();
+        const float inv = 1.f / l;
+        const int row = qb * kBM + r;
+        uint4* orow = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * p.N + row) * D);
+        const float* dvp = p.dv + static_cast<size_t>(zkv) * D;
+#pragma unroll 1
+        for (int cb = 0; cb < D / 32; ++cb) {
+          uint32_t o[32];
+          SAGE_TMEM_LD32(tO + cb * 32, o);
+          tmem_wait_ld();
+          uint32_t hv[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float x0 = __uint_as_float(o[2 * i]) * inv;
+            float x1 = __uint_as_float(o[2 * i + 1]) * inv;
+            if (VAR == 1) {
+              x0 *= dvp[cb * 32 + 2 * i];
+              x1 *= dvp[cb * 32 + 2 * i + 1];
+            }
+            hv[i] = pack_f16x2(x0, x1);
+          }
+          if (row < p.N) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              orow[cb * 4 + i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 3-D map over [slabs][N][d] of `elem`-byte elements, box = box_inner x 128 x 1.
+static bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem, int d,
+                     int N, int slabs, int box_inner, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(slabs)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem,
+                                 static_cast<cuuint64_t>(N) * d * elem};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 128u, 1u};
+  const cuuint32_t es[3] = {1u, 1u, 1u};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <int D, int VAR, bool CAUSAL>
+static cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
+  using C = Cfg<D, VAR>;
+  static bool attr_set = false;
+  auto kern = k_attn<D, VAR, CAUSAL>;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  CUtensorMap tq, tk, tv;
+  const CUtensorMapSwizzle qk_sw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  bool ok = make_map(&tq, a.q_hat, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, a.N, a.B * a.H, D, qk_sw) &&
+            make_map(&tk, a.k_hat, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, a.N, a.B * a.H_kv, D, qk_sw);
+  if (VAR == 0)
+    ok = ok && make_map(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, D, a.N, a.B * a.H_kv, 64,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    ok = ok && make_map(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, a.N, a.B * a.H_kv, D, qk_sw);
+  if (!ok) return cudaErrorInvalidValue;
+  AttnKParams kp;
+  kp.dq = a.delta_q;
+  kp.dk = a.delta_k;
+  kp.dv = a.delta_v;
+  kp.o = static_cast<__half*>(a.o);
+  kp.H = a.H;
+  kp.Hkv = a.H_kv;
+  kp.N = a.N;
+  kp.nqb = (a.N + kBM - 1) / kBM;
+  kp.nkvb = (a.N + kBN - 1) / kBN;
+  kp.timeout_ns = a.timeout_ns;
+  dim3 grid((kp.nqb + 1) / 2, a.B * a.H);
+  kern<<<grid, kAttnThreads, C::SMEM, st>>>(tq, tk, tv, kp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
+  const bool c = a.causal != 0;
+  if (a.d == 128) {
+    if (a.variant == 0) return c ? launch_t<128, 0, true>(a, st) : launch_t<128, 0, false>(a, st);
+    return c ? launch_t<128, 1, true>(a, st) : launch_t<128, 1, false>(a, st);
+  }
+  if (a.variant == 0) return c ? launch_t<64, 0, true>(a, st) : launch_t<64, 0, false>(a, st);
+  return c ? launch_t<64, 1, true>(a, st) : launch_t<64, 1, false>(a, st);
+}
+
+// ---------------------------------------------------------------- failure-detection self-test
+__global__ void k_selftest_wait(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // nothing ever arrives on `bar`: the bounded wait must give up
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, reinterpret_cast<volatile int*>(&abort_flag), timeout_ns, 0xEEu);
+}
+
+cudaError_t launch_selftest_wait(uint64_t timeout_ns, cudaStream_t st) {
+  k_selftest_wait<<<1, 32, 0, st>>>(timeout_ns);
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_error(uint32_t* word) {
+  uint32_t w = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w));
+  if (e != cudaSuccess) return e;
+  if (w != 0) e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
+  *word = w;
+  return e;
+}
+
+}  // namespace sage

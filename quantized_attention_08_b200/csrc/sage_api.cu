@@ -1,0 +1,380 @@
+// sage_api.cu -- the C ABI declared in include/sage.h: argument checks,
+// workspace carving, stream-ordered allocation and kernel launches.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+
+#include "../../include/sage.h"
+#include "sage_internal.h"
+
+namespace {
+
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+
+constexpr int kMaxDevices = 64;
+int g_dev_ok[kMaxDevices];  // 0 unknown, 1 sm_100, -1 other
+
+sage_status_t check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SAGE_ERR_DEVICE;
+  if (g_dev_ok[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return SAGE_ERR_CUDA;
+    g_dev_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  return g_dev_ok[dev] == 1 ? SAGE_OK : SAGE_ERR_DEVICE;
+}
+
+bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool a4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+sage_status_t check_sizes(int B, int H, int H_kv, int N, int d) {
+  if (B < 0 || H <= 0 || H_kv <= 0 || N < 0) return SAGE_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
+  if (H % H_kv != 0) return SAGE_ERR_UNSUPPORTED;
+  // grid.y = B*H; TMA coordinates are 32-bit
+  if (static_cast<long long>(B) * H > 65535) return SAGE_ERR_UNSUPPORTED;
+  if (N > (1 << 24)) return SAGE_ERR_UNSUPPORTED;
+  return SAGE_OK;
+}
+
+sage_status_t from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return SAGE_OK;
+  if (e == cudaErrorMemoryAllocation) return SAGE_ERR_NO_MEMORY;
+  return SAGE_ERR_CUDA;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Layout of the intermediates inside one workspace.
+struct WsLayout {
+  size_t q_hat, k_hat, v_hat, delta_q, delta_k, mean_k, delta_v, ksum, vmax, total;
+};
+
+WsLayout ws_layout(int B, int H, int H_kv, int N, int d, int variant) {
+  WsLayout L;
+  const size_t nb = static_cast<size_t>((N + 127) / 128);
+  const size_t nq = static_cast<size_t>(B) * H, nk = static_cast<size_t>(B) * H_kv;
+  const size_t nchunk = sage::stat_chunks(N);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  L.q_hat = take(nq * N * d);
+  L.k_hat = take(nk * N * d);
+  L.v_hat = take(variant == SAGE_VARIANT_8P8 ? nk * N * d : 0);
+  L.delta_q = take(nq * nb * 4);
+  L.delta_k = take(nk * nb * 4);
+  L.mean_k = take(nk * d * 4);
+  L.delta_v = take(variant == SAGE_VARIANT_8P8 ? nk * d * 4 : 0);
+  L.ksum = take(nk * nchunk * d * 8);
+  L.vmax = take(variant == SAGE_VARIANT_8P8 ? nk * nchunk * d * 4 : 0);
+  L.total = off;
+  return L;
+}
+
+// The whole pass with intermediates carved from `ws` (L.total bytes).
+sage_status_t run_forward(const void* q, const void* k, const void* v, void* o, int B, int H,
+                          int H_kv, int N, int d, int causal, float sm_scale, int variant,
+                          uint8_t* ws, const WsLayout& L, cudaStream_t st) {
+  const bool v8 = variant == SAGE_VARIANT_8P8;
+  const int slabs = B * H_kv;
+  int8_t* q_hat = reinterpret_cast<int8_t*>(ws + L.q_hat);
+  int8_t* k_hat = reinterpret_cast<int8_t*>(ws + L.k_hat);
+  uint8_t* v_hat = v8 ? ws + L.v_hat : nullptr;
+  float* delta_q = reinterpret_cast<float*>(ws + L.delta_q);
+  float* delta_k = reinterpret_cast<float*>(ws + L.delta_k);
+  float* mean_k = reinterpret_cast<float*>(ws + L.mean_k);
+  float* delta_v = v8 ? reinterpret_cast<float*>(ws + L.delta_v) : nullptr;
+  long long* ksum = reinterpret_cast<long long*>(ws + L.ksum);
+  uint32_t* vmax = v8 ? reinterpret_cast<uint32_t*>(ws + L.vmax) : nullptr;
+
+  cudaError_t e = sage::launch_colstats(k, v8 ? v : nullptr, slabs, N, d, ksum, vmax, st);
+  if (e == cudaSuccess)
+    e = sage::launch_finalize(ksum, vmax, slabs, N, d, 448.0f, mean_k, delta_v, st);
+  if (e == cudaSuccess) {
+    sage::QuantArgs qa;
+    qa.q = q;
+    qa.k = k;
+    qa.v = v8 ? v : nullptr;
+    qa.q_hat = q_hat;
+    qa.k_hat = k_hat;
+    qa.v_hat = v_hat;
+    qa.delta_q = delta_q;
+    qa.delta_k = delta_k;
+    qa.mean_k = mean_k;
+    qa.delta_v = delta_v;
+    qa.sm_scale = sm_scale;
+    qa.B = B;
+    qa.H = H;
+    qa.H_kv = H_kv;
+    qa.N = N;
+    qa.d = d;
+    e = sage::launch_quant(qa, st);
+  }
+  if (e == cudaSuccess) {
+    sage::AttnArgs aa;
+    aa.q_hat = q_hat;
+    aa.k_hat = k_hat;
+    aa.delta_q = delta_q;
+    aa.delta_k = delta_k;
+    aa.v = v8 ? static_cast<const void*>(v_hat) : v;
+    aa.delta_v = delta_v;
+    aa.o = o;
+    aa.B = B;
+    aa.H = H;
+    aa.H_kv = H_kv;
+    aa.N = N;
+    aa.d = d;
+    aa.causal = causal;
+    aa.variant = variant;
+    aa.timeout_ns = g_timeout_ns.load();
+    e = sage::launch_attention(aa, st);
+  }
+  return from_cuda(e);
+}
+
+sage_status_t check_fwd_args(const void* q, const void* k, const void* v, void* o, int B, int H,
+                             int H_kv, int N, int d, int causal, float sm_scale, int variant) {
+  sage_status_t s = check_sizes(B, H, H_kv, N, d);
+  if (s != SAGE_OK) return s;
+  if (variant != SAGE_VARIANT_B && variant != SAGE_VARIANT_8P8) return SAGE_ERR_UNSUPPORTED;
+  if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return SAGE_OK;
+  if (!q || !k || !v || !o) return SAGE_ERR_INVALID_ARG;
+  if (!a16(q) || !a16(k) || !a16(v) || !a16(o)) return SAGE_ERR_MISALIGNED;
+  return SAGE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sage_status_t sage_smooth_quant_qk(const void* q, const void* k, int B, int H, int H_kv, int N,
+                                   int d, float sm_scale, int8_t* q_hat, int8_t* k_hat,
+                                   float* delta_q, float* delta_k, float* mean_k, void* stream) {
+  sage_status_t s = check_sizes(B, H, H_kv, N, d);
+  if (s != SAGE_OK) return s;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return SAGE_OK;
+  if (!q || !k || !q_hat || !k_hat || !delta_q || !delta_k || !mean_k) return SAGE_ERR_INVALID_ARG;
+  if (!a16(q) || !a16(k) || !a16(q_hat) || !a16(k_hat) || !a4(delta_q) || !a4(delta_k) ||
+      !a4(mean_k))
+    return SAGE_ERR_MISALIGNED;
+  if ((s = check_device()) != SAGE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int slabs = B * H_kv;
+  const size_t bytes = static_cast<size_t>(slabs) * sage::stat_chunks(N) * d * 8;
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocAsync(&scratch, bytes, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  long long* ksum = static_cast<long long*>(scratch);
+  e = sage::launch_colstats(k, nullptr, slabs, N, d, ksum, nullptr, st);
+  if (e == cudaSuccess) e = sage::launch_finalize(ksum, nullptr, slabs, N, d, 0.f, mean_k, nullptr, st);
+  if (e == cudaSuccess) {
+    sage::QuantArgs qa;
+    std::memset(&qa, 0, sizeof(qa));
+    qa.q = q;
+    qa.k = k;
+    qa.q_hat = q_hat;
+    qa.k_hat = k_hat;
+    qa.delta_q = delta_q;
+    qa.delta_k = delta_k;
+    qa.mean_k = mean_k;
+    qa.sm_scale = sm_scale;
+    qa.B = B;
+    qa.H = H;
+    qa.H_kv = H_kv;
+    qa.N = N;
+    qa.d = d;
+    e = sage::launch_quant(qa, st);
+  }
+  cudaError_t ef = cudaFreeAsync(scratch, st);
+  return from_cuda(e != cudaSuccess ? e : ef);
+}
+
+sage_status_t sage_quant_v_fp8(const void* v, int B, int H_kv, int N, int d, float v_r,
+                               uint8_t* v_hat, float* delta_v, void* stream) {
+  sage_status_t s = check_sizes(B, H_kv, H_kv, N, d);
+  if (s != SAGE_OK) return s;
+  if (!(v_r > 0.f) || !(v_r <= 448.f)) return SAGE_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return SAGE_OK;
+  if (!v || !v_hat || !delta_v) return SAGE_ERR_INVALID_ARG;
+  if (!a16(v) || !a16(v_hat) || !a4(delta_v)) return SAGE_ERR_MISALIGNED;
+  if ((s = check_device()) != SAGE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int slabs = B * H_kv;
+  const size_t bytes = static_cast<size_t>(slabs) * sage::stat_chunks(N) * d * 4;
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocAsync(&scratch, bytes, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  uint32_t* vmax = static_cast<uint32_t*>(scratch);
+  e = sage::launch_colstats(nullptr, v, slabs, N, d, nullptr, vmax, st);
+  if (e == cudaSuccess) e = sage::launch_finalize(nullptr, vmax, slabs, N, d, v_r, nullptr, delta_v, st);
+  if (e == cudaSuccess) {
+    sage::QuantArgs qa;
+    std::memset(&qa, 0, sizeof(qa));
+    qa.v = v;
+    qa.v_hat = v_hat;
+    qa.delta_v = delta_v;
+    qa.B = B;
+    qa.H = H_kv;
+    qa.H_kv = H_kv;
+    qa.N = N;
+    qa.d = d;
+    e = sage::launch_quant(qa, st);
+  }
+  cudaError_t ef = cudaFreeAsync(scratch, st);
+  return from_cuda(e != cudaSuccess ? e : ef);
+}
+
+sage_status_t sage_attn_fwd_quantized(const int8_t* q_hat, const int8_t* k_hat,
+                                      const float* delta_q, const float* delta_k,
+                                      const void* v_or_vhat, const float* delta_v, void* o, int B,
+                                      int H, int H_kv, int N, int d, int causal, int variant,
+                                      void* stream) {
+  sage_status_t s = check_sizes(B, H, H_kv, N, d);
+  if (s != SAGE_OK) return s;
+  if (variant != SAGE_VARIANT_B && variant != SAGE_VARIANT_8P8) return SAGE_ERR_UNSUPPORTED;
+  if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return SAGE_OK;
+  if (!q_hat || !k_hat || !delta_q || !delta_k || !v_or_vhat || !o) return SAGE_ERR_INVALID_ARG;
+  if (variant == SAGE_VARIANT_8P8 && !delta_v) return SAGE_ERR_INVALID_ARG;
+  if (!a16(q_hat) || !a16(k_hat) || !a16(v_or_vhat) || !a16(o) || !a4(delta_q) || !a4(delta_k) ||
+      (delta_v && !a4(delta_v)))
+    return SAGE_ERR_MISALIGNED;
+  if ((s = check_device()) != SAGE_OK) return s;
+  sage::AttnArgs aa;
+  aa.q_hat = q_hat;
+  aa.k_hat = k_hat;
+  aa.delta_q = delta_q;
+  aa.delta_k = delta_k;
+  aa.v = v_or_vhat;
+  aa.delta_v = delta_v;
+  aa.o = o;
+  aa.B = B;
+  aa.H = H;
+  aa.H_kv = H_kv;
+  aa.N = N;
+  aa.d = d;
+  aa.causal = causal;
+  aa.variant = variant;
+  aa.timeout_ns = g_timeout_ns.load();
+  return from_cuda(sage::launch_attention(aa, static_cast<cudaStream_t>(stream)));
+}
+
+size_t sage_attn_workspace_bytes(int B, int H, int H_kv, int N, int d, int variant) {
+  if (check_sizes(B, H, H_kv, N, d) != SAGE_OK || B == 0 || N == 0) return 0;
+  return ws_layout(B, H, H_kv, N, d, variant).total;
+}
+
+sage_status_t sage_attn_fwd_ws(const void* q, const void* k, const void* v, void* o, int B, int H,
+                               int H_kv, int N, int d, int causal, float sm_scale, int variant,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  sage_status_t s = check_fwd_args(q, k, v, o, B, H, H_kv, N, d, causal, sm_scale, variant);
+  if (s != SAGE_OK || B == 0 || N == 0) return s;
+  if ((s = check_device()) != SAGE_OK) return s;
+  const WsLayout L = ws_layout(B, H, H_kv, N, d, variant);
+  if (workspace == nullptr || ws_bytes < L.total) return SAGE_ERR_NO_MEMORY;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SAGE_ERR_MISALIGNED;
+  return run_forward(q, k, v, o, B, H, H_kv, N, d, causal, sm_scale, variant,
+                     static_cast<uint8_t*>(workspace), L, static_cast<cudaStream_t>(stream));
+}
+
+sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H,
+                            int H_kv, int N, int d, int causal, float sm_scale, int variant,
+                            void* stream) {
+  sage_status_t s = check_fwd_args(q, k, v, o, B, H, H_kv, N, d, causal, sm_scale, variant);
+  if (s != SAGE_OK || B == 0 || N == 0) return s;
+  if ((s = check_device()) != SAGE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(B, H, H_kv, N, d, variant);
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, L.total, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  s = run_forward(q, k, v, o, B, H, H_kv, N, d, causal, sm_scale, variant,
+                  static_cast<uint8_t*>(ws), L, st);
+  cudaError_t ef = cudaFreeAsync(ws, st);
+  if (s != SAGE_OK) return s;
+  return from_cuda(ef);
+}
+
+sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                                 void* o_host, int B, int H, int H_kv, int N, int d, int causal,
+                                 float sm_scale, int variant, void* stream) {
+  sage_status_t s = check_sizes(B, H, H_kv, N, d);
+  if (s != SAGE_OK) return s;
+  if (variant != SAGE_VARIANT_B && variant != SAGE_VARIANT_8P8) return SAGE_ERR_UNSUPPORTED;
+  if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return SAGE_OK;
+  if (!q_host || !k_host || !v_host || !o_host) return SAGE_ERR_INVALID_ARG;
+  if ((s = check_device()) != SAGE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t qb = static_cast<size_t>(B) * H * N * d * 2;
+  const size_t kb = static_cast<size_t>(B) * H_kv * N * d * 2;
+  const WsLayout L = ws_layout(B, H, H_kv, N, d, variant);
+  const size_t off_k = align256(qb), off_v = off_k + align256(kb), off_o = off_v + align256(kb);
+  const size_t off_ws = off_o + align256(qb);
+  void* buf = nullptr;
+  cudaError_t e = cudaMallocAsync(&buf, off_ws + L.total, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  uint8_t* base = static_cast<uint8_t*>(buf);
+  e = cudaMemcpyAsync(base, q_host, qb, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(base + off_k, k_host, kb, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(base + off_v, v_host, kb, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) {
+    s = run_forward(base, base + off_k, base + off_v, base + off_o, B, H, H_kv, N, d, causal,
+                    sm_scale, variant, base + off_ws, L, st);
+    if (s == SAGE_OK)
+      e = cudaMemcpyAsync(o_host, base + off_o, qb, cudaMemcpyDeviceToHost, st);
+  }
+  cudaError_t ef = cudaFreeAsync(buf, st);
+  cudaError_t es = cudaStreamSynchronize(st);
+  if (s != SAGE_OK) return s;
+  if (e != cudaSuccess) return from_cuda(e);
+  if (ef != cudaSuccess) return from_cuda(ef);
+  return from_cuda(es);
+}
+
+int sage_v_hat_layout(void) { return 0; }
+
+sage_status_t sage_get_device_error(void* stream, uint32_t* detail) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SAGE_ERR_CUDA;
+  uint32_t w = 0;
+  if (sage::read_and_clear_error(&w) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (detail) *detail = w;
+  return (w & sage::ERR_TIMEOUT) ? SAGE_ERR_DEVICE_TIMEOUT : SAGE_OK;
+}
+
+void sage_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns == 0 ? 1 : ns); }
+
+sage_status_t sage_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
+  sage_status_t s = check_device();
+  if (s != SAGE_OK) return s;
+  return from_cuda(sage::launch_selftest_wait(timeout_ns, static_cast<cudaStream_t>(stream)));
+}
+
+const char* sage_status_string(sage_status_t status) {
+  switch (status) {
+    case SAGE_OK: return "ok";
+    case SAGE_ERR_INVALID_ARG: return "invalid argument";
+    case SAGE_ERR_UNSUPPORTED: return "unsupported shape or variant";
+    case SAGE_ERR_MISALIGNED: return "pointer not aligned";
+    case SAGE_ERR_DEVICE: return "current device is not a B200 (compute capability 10.0)";
+    case SAGE_ERR_CUDA: return "CUDA call failed";
+    case SAGE_ERR_DEVICE_TIMEOUT: return "a kernel abandoned a bounded wait";
+    case SAGE_ERR_NO_MEMORY: return "out of device memory or workspace too small";
+  }
+  return "unknown status";
+}
+
+const char* sage_version(void) { return "0.1.0"; }
+
+}  // extern "C"

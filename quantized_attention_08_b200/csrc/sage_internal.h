@@ -1,0 +1,53 @@
+// sage_internal.h -- declarations shared by the library's translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "sage_ptx.cuh"
+
+namespace sage {
+
+struct QuantArgs {
+  const void* q;        // fp16 [B,H,N,d] or nullptr
+  const void* k;        // fp16 [B,Hkv,N,d] or nullptr
+  const void* v;        // fp16 [B,Hkv,N,d] or nullptr (8+8 only)
+  int8_t* q_hat;
+  int8_t* k_hat;
+  uint8_t* v_hat;
+  float* delta_q;
+  float* delta_k;
+  const float* mean_k;
+  const float* delta_v;
+  float sm_scale;
+  int B, H, H_kv, N, d;
+};
+
+size_t stat_chunks(int N);
+cudaError_t launch_colstats(const void* k, const void* v, int slabs, int N, int D, long long* ksum,
+                            uint32_t* vmax, cudaStream_t st);
+cudaError_t launch_finalize(const long long* ksum, const uint32_t* vmax, int slabs, int N, int D,
+                            float v_r, float* mean_k, float* delta_v, cudaStream_t st);
+cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st);
+
+struct AttnArgs {
+  const int8_t* q_hat;
+  const int8_t* k_hat;
+  const float* delta_q;
+  const float* delta_k;
+  const void* v;         // fp16 V (variant B) or e4m3 codes (8+8)
+  const float* delta_v;  // 8+8 only
+  void* o;               // fp16 [B,H,N,d]
+  int B, H, H_kv, N, d, causal, variant;
+  uint64_t timeout_ns;
+};
+
+// Returns a cudaError_t; CUDA_ERROR codes of tensor-map encoding are mapped
+// to cudaErrorInvalidValue.
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st);
+
+cudaError_t launch_selftest_wait(uint64_t timeout_ns, cudaStream_t st);
+cudaError_t read_and_clear_error(uint32_t* word);
+
+}  // namespace sage

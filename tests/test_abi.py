@@ -1,0 +1,95 @@
+"""CPU checks of the C-ABI library: it builds, loads without a GPU, and
+exports every function declared in include/sage.h; host-side argument
+checks that return before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sage.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from quantized_attention_08_b200 import build
+    build.build()
+    import quantized_attention_08_b200 as pkg
+    return pkg.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+(sage_[a-z0-9_]+)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("sage_smooth_quant_qk", "sage_quant_v_fp8", "sage_attn_fwd",
+              "sage_attn_fwd_quantized", "sage_get_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_covers_every_declared_symbol():
+    import quantized_attention_08_b200 as pkg
+    for name in declared_functions():
+        assert name in pkg._SIGS, name
+        assert callable(getattr(pkg, name)), name
+
+
+def test_status_strings_and_version(lib):
+    import quantized_attention_08_b200 as pkg
+    assert pkg.sage_status_string(0) == "ok"
+    assert "aligned" in pkg.sage_status_string(3)
+    assert re.match(r"\d+\.\d+\.\d+", pkg.sage_version())
+    assert pkg.sage_v_hat_layout() == 0
+
+
+def test_host_argument_checks_need_no_gpu(lib):
+    """Shape / variant / scale errors are reported before any CUDA call."""
+    f = lib.sage_attn_fwd
+    fake = ctypes.c_void_p(1 << 20)
+    # d = 96 unsupported
+    assert f(fake, fake, fake, fake, 1, 2, 2, 128, 96, 0, 0.1, 0, None) == 2
+    # H not a multiple of H_kv
+    assert f(fake, fake, fake, fake, 1, 3, 2, 128, 64, 0, 0.1, 0, None) == 2
+    # unknown variant
+    assert f(fake, fake, fake, fake, 1, 2, 2, 128, 64, 0, 0.1, 7, None) == 2
+    # sm_scale <= 0, NaN
+    assert f(fake, fake, fake, fake, 1, 2, 2, 128, 64, 0, 0.0, 0, None) == 1
+    assert f(fake, fake, fake, fake, 1, 2, 2, 128, 64, 0, float("nan"), 0, None) == 1
+    # negative size, bad causal flag
+    assert f(fake, fake, fake, fake, 1, 2, 2, -1, 64, 0, 0.1, 0, None) == 1
+    assert f(fake, fake, fake, fake, 1, 2, 2, 128, 64, 2, 0.1, 0, None) == 1
+    # null pointer
+    assert f(None, fake, fake, fake, 1, 2, 2, 128, 64, 0, 0.1, 0, None) == 1
+    # misaligned
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert f(odd, fake, fake, fake, 1, 2, 2, 128, 64, 0, 0.1, 0, None) == 3
+    # empty problems are a no-op
+    assert f(None, None, None, None, 0, 2, 2, 128, 64, 0, 0.1, 0, None) == 0
+    assert f(None, None, None, None, 1, 2, 2, 0, 64, 0, 0.1, 0, None) == 0
+    # V range of the fp8 quantizer
+    g = lib.sage_quant_v_fp8
+    assert g(fake, 1, 2, 128, 64, 500.0, fake, fake, None) == 1
+    assert g(fake, 1, 2, 128, 64, 0.0, fake, fake, None) == 1
+
+
+def test_workspace_size_is_consistent(lib):
+    import quantized_attention_08_b200 as pkg
+    a = pkg.sage_attn_workspace_bytes(1, 32, 8, 8192, 128, "B")
+    b = pkg.sage_attn_workspace_bytes(1, 32, 8, 8192, 128, "8+8")
+    # q_hat + k_hat at least, and 8+8 adds v_hat
+    assert a >= 32 * 8192 * 128 + 8 * 8192 * 128
+    assert b >= a + 8 * 8192 * 128
+    assert pkg.sage_attn_workspace_bytes(0, 32, 8, 8192, 128, "B") == 0
+    assert pkg.sage_attn_workspace_bytes(1, 32, 8, 8192, 96, "B") == 0
