@@ -170,6 +170,11 @@ void sage_set_wait_timeout_ns(uint64_t ns);
  */
 sage_status_t sage_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
 
+/* Description of the step that last failed in this thread (for SAGE_ERR_CUDA
+ * and friends): the CUDA call, its error string and code.  "none" if no
+ * failure was recorded.  The pointer stays valid until the thread's next call. */
+const char* sage_last_error_detail(void);
+
 /* Static description of a status code. */
 const char* sage_status_string(sage_status_t status);
 

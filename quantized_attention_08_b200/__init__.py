@@ -47,6 +47,7 @@ _SIGS = {
     "sage_selftest_wait_timeout": (_i, [_c.c_uint64, _vp]),
     "sage_status_string": (_c.c_char_p, [_i]),
     "sage_version": (_c.c_char_p, []),
+    "sage_last_error_detail": (_c.c_char_p, []),
 }
 
 _lib_handle = None
@@ -72,7 +73,12 @@ def load_library() -> ctypes.CDLL:
 class SageError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {sage_status_string(status)} (status {status})")
+        super().__init__(f"{where}: {sage_status_string(status)} (status {status}); "
+                         f"last failing step: {sage_last_error_detail()}")
+
+
+def sage_last_error_detail() -> str:
+    return load_library().sage_last_error_detail().decode()
 
 
 def sage_status_string(status: int) -> str:

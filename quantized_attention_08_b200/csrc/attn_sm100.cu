@@ -25,6 +25,7 @@
 // tensor memory and exits.
 #include <cuda_fp16.h>
 #include <math.h>
+#include <stdio.h>
 
 #include "sage_internal.h"
 
@@ -128,7 +129,8 @@ __device__ __forceinline__ float softmax_tile(uint32_t (&a)[128], float c, float
 }
 
 template <int D, int VAR, bool CAUSAL>
-__global__ void __maxnreg__(200)
+// 10 warps: up to 3 share one SM sub-partition's 16K registers -> <= 168 per thread.
+__global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, const AttnKParams p) {
   using C = Cfg<D, VAR>;
@@ -401,7 +403,7 @@ static EncodeTiledFn encode_fn() {
 }
 
 // 3-D map over [slabs][N][d] of `elem`-byte elements, box = box_inner x 128 x 1.
-static bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem, int d,
+static bool make_map_impl(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem, int d,
                      int N, int slabs, int box_inner, CUtensorMapSwizzle sw) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
@@ -411,9 +413,20 @@ static bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, i
                                  static_cast<cuuint64_t>(N) * d * elem};
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 128u, 1u};
   const cuuint32_t es[3] = {1u, 1u, 1u};
-  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
+  const CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) set_error_detail("cuTensorMapEncodeTiled", cudaErrorInvalidValue, static_cast<int>(r));
+  return r == CUDA_SUCCESS;
+}
+
+static bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem, int d,
+                     int N, int slabs, int box_inner, CUtensorMapSwizzle sw) {
+  if (encode_fn() == nullptr) {
+    set_error_detail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorInvalidValue);
+    return false;
+  }
+  return make_map_impl(m, base, dt, elem, d, N, slabs, box_inner, sw);
 }
 
 template <int D, int VAR, bool CAUSAL>
@@ -423,7 +436,10 @@ static cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   auto kern = k_attn<D, VAR, CAUSAL>;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+      set_error_detail("cudaFuncSetAttribute(attention)", e, C::SMEM);
+      return e;
+    }
     attr_set = true;
   }
   CUtensorMap tq, tk, tv;
@@ -449,7 +465,9 @@ static cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   kp.timeout_ns = a.timeout_ns;
   dim3 grid((kp.nqb + 1) / 2, a.B * a.H);
   kern<<<grid, kAttnThreads, C::SMEM, st>>>(tq, tk, tv, kp);
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) set_error_detail("attention kernel launch", e, C::SMEM);
+  return e;
 }
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
@@ -480,6 +498,14 @@ cudaError_t launch_selftest_wait(uint64_t timeout_ns, cudaStream_t st) {
   k_selftest_wait<<<1, 32, 0, st>>>(timeout_ns);
   return cudaGetLastError();
 }
+
+static thread_local char t_detail[256] = "none";
+
+void set_error_detail(const char* step, cudaError_t e, int extra) {
+  snprintf(t_detail, sizeof(t_detail), "%s: %s (%d) [%d]", step, cudaGetErrorString(e),
+           static_cast<int>(e), extra);
+}
+const char* error_detail() { return t_detail; }
 
 cudaError_t read_and_clear_error(uint32_t* word) {
   uint32_t w = 0, zero = 0;

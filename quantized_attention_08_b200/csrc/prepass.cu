@@ -286,14 +286,18 @@ cudaError_t launch_colstats(const void* k, const void* v, int slabs, int N, int 
   else
     k_colstats<64><<<grid, kThreads, 0, st>>>(static_cast<const uint4*>(k),
                                               static_cast<const uint4*>(v), N, nchunk, ksum, vmax);
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) set_error_detail("column statistics kernel launch", e);
+  return e;
 }
 
 cudaError_t launch_finalize(const long long* ksum, const uint32_t* vmax, int slabs, int N, int D,
                             float v_r, float* mean_k, float* delta_v, cudaStream_t st) {
   const int nchunk = static_cast<int>(stat_chunks(N));
   k_finalize<<<slabs, D, 0, st>>>(ksum, vmax, nchunk, D, N, v_r, mean_k, delta_v);
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) set_error_detail("finalize kernel launch", e);
+  return e;
 }
 
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st) {
@@ -320,7 +324,9 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st) {
     k_quant<128><<<total, kThreads, 0, st>>>(J);
   else
     k_quant<64><<<total, kThreads, 0, st>>>(J);
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) set_error_detail("quantization kernel launch", e);
+  return e;
 }
 
 }  // namespace sage

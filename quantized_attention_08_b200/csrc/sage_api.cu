@@ -297,7 +297,10 @@ sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* o
   const WsLayout L = ws_layout(B, H, H_kv, N, d, variant);
   void* ws = nullptr;
   cudaError_t e = cudaMallocAsync(&ws, L.total, st);
-  if (e != cudaSuccess) return from_cuda(e);
+  if (e != cudaSuccess) {
+    sage::set_error_detail("cudaMallocAsync(workspace)", e);
+    return from_cuda(e);
+  }
   s = run_forward(q, k, v, o, B, H, H_kv, N, d, causal, sm_scale, variant,
                   static_cast<uint8_t*>(ws), L, st);
   cudaError_t ef = cudaFreeAsync(ws, st);
@@ -376,5 +379,7 @@ const char* sage_status_string(sage_status_t status) {
 }
 
 const char* sage_version(void) { return "0.1.0"; }
+
+const char* sage_last_error_detail(void) { return sage::error_detail(); }
 
 }  // extern "C"

@@ -50,4 +50,9 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t timeout_ns, cudaStream_t st);
 cudaError_t read_and_clear_error(uint32_t* word);
 
+// Records a human-readable description of the last failing step of this
+// thread's most recent call (see sage_last_error_detail()).
+void set_error_detail(const char* step, cudaError_t e, int extra = 0);
+const char* error_detail();
+
 }  // namespace sage
