@@ -1,0 +1,368 @@
+"""Throughput of the SageAttention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--variant B|8+8] [--impl sage|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+the pre-pass (Smooth K, INT8 quantization of Q*sm_scale and K, E4M3
+quantization of V for 8+8) followed by the attention kernel.  The default
+workload is the video-DiT shape (B=1, H=24, N=32768, d=128, non-causal, 8+8),
+the configuration the headline metric is quoted on.
+
+Metric: TOPS = 4*B*H*N^2*d / t (halved for causal), whole-job over all ranks.
+`--impl reference` times the CPU oracle (numpy) on the host cores instead.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs an independent
+replica of the workload on its own GPU (the path shards by (batch, kv-head)
+group with no exchange), so scaling is weak; the only collectives are the
+timing barrier and the max-over-ranks of the elapsed time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+DEFAULT_WORKLOAD = "video_dit_h24_n32768_d128"
+SPEC_8BIT_TOPS = 4500.0          # B200 dense INT8 / FP8 tensor peak, NVIDIA spec
+NOMINAL_8BIT_OVER_BF16 = 2.0     # 4.5 / 2.25 PFLOP/s dense
+
+# DRAM traffic per attention launch from an ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum), keyed by the attention source hash it was taken on;
+# reported as null once the kernel source changes.
+NCU_TRAFFIC = {
+    # 639.3 MB measured on B=8,H=16,N=8192 (8+8), scaled by elements per tensor
+    # (attention DRAM traffic is linear in B*H*N*d once K/V re-reads hit L2)
+    ("950264ac83e970ff", "video_dit_h24_n32768_d128", "8+8"): 479.6e6,
+}
+
+
+def _src_hash() -> str:
+    p = os.path.join(ROOT, "quantized_attention_08_b200", "csrc", "attn_sm100.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def _peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except OSError:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (getattr(self, "out", "") or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i] == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+class OracleSampler:
+    """Times the CPU oracle on bounded samples of workload `w`.
+
+    The pre-pass (Smooth K and the quantizers) of one (batch, head) slab is
+    timed once; a sample is then the oracle's attention for some q blocks of
+    that head against all keys (all causal-visible keys), charged with its
+    share rows/N of the pre-pass time.  Throughput = 4*rows*keys*d / time."""
+
+    def __init__(self, w, variant):
+        import oracle
+        self.oracle, self.w, self.variant = oracle, w, variant
+        q, k, v = workloads.generate(w.with_(B=1, H=1, H_kv=1))
+        t0 = time.perf_counter()
+        self.qh, self.dq = oracle.quant_q(q, w.scale)
+        self.kh, self.dk, _ = oracle.smooth_quant_k(k)
+        if variant == "8+8":
+            vh, self.dv = oracle.quant_v_fp8(v)
+            self.vop, self.operand = oracle.e4m3_decode(vh), "e4m3"
+        else:
+            self.vop, self.dv, self.operand = v, None, "fp16"
+        self.t_prepass = time.perf_counter() - t0
+        self.nqb = (w.N + 127) // 128
+        self.next = 0
+        try:
+            from threadpoolctl import threadpool_info
+            self.threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+        except Exception:  # noqa: BLE001
+            self.threads = os.cpu_count() or 1
+
+    def sample(self, budget_s: float):
+        w = self.w
+        ops, t, blocks = 0.0, 0.0, 0
+        while blocks == 0 or t < budget_s:
+            qb = (self.next * 37) % self.nqb      # spread over the sequence
+            self.next += 1
+            t0 = time.perf_counter()
+            self.oracle.attention_online(self.qh, self.kh, self.dq, self.dk, self.vop,
+                                         causal=w.causal, operand=self.operand, dv=self.dv,
+                                         q_blocks=[qb])
+            rows = min(128, w.N - qb * 128)
+            t += time.perf_counter() - t0 + self.t_prepass * rows / w.N
+            keys = w.N
+            if w.causal:
+                keys = (qb * 128 + (rows + 1) / 2.0)   # mean visible keys of the block's rows
+            ops += 4.0 * rows * keys * w.d
+            blocks += 1
+        desc = (f"oracle (numpy fp64) quantized mirror, {blocks} q block(s) x 128 rows of one head "
+                f"against all keys (N={w.N}), plus that head's pre-pass pro rata "
+                f"({self.t_prepass:.2f} s per head); {t:.1f} s")
+        return ops / t, desc
+
+
+def run_reference(args, w, variant):
+    """--impl reference: the CPU oracle, timed on the host cores, each step a
+    bounded sample sized so that the whole run takes a few minutes."""
+    smp = OracleSampler(w, variant)
+    budget = max(0.2, min(args.ref_budget, 150.0 / (args.steps + args.warmup)))
+    per_step, desc = [], ""
+    for s in range(args.warmup + args.steps):
+        ops_s, desc = smp.sample(budget)
+        if s >= args.warmup:
+            per_step.append(ops_s)
+    value = statistics.median(per_step) / 1e12
+    line = {
+        "impl": "reference", "metric": "quantized attention TOPS (4BHN^2d/t) at N=32K d=128; % of B200 INT8/FP8 tensor peak",
+        "value": value, "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy, workload recipe; no dataset)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N, "d": w.d,
+                   "causal": w.causal, "variant": variant},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": smp.threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--variant", default=None)
+    ap.add_argument("--impl", default="sage", choices=["sage", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    w = workloads.get(args.workload)
+    variant = args.variant or w.variants[-1]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, w, variant)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import quantized_attention_08_b200 as sage
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    sage.load_library()
+
+    q, k, v = workloads.generate(w)
+    tq, tk, tv = (torch.from_numpy(x).to(dev) for x in (q, k, v))
+    B, H, N, d = q.shape
+    Hk = k.shape[1]
+    v8 = variant == "8+8"
+    nb = (N + 127) // 128
+    outs = (torch.empty_like(tq, dtype=torch.int8), torch.empty_like(tk, dtype=torch.int8),
+            torch.empty(B, H, nb, dtype=torch.float32, device=dev),
+            torch.empty(B, Hk, nb, dtype=torch.float32, device=dev),
+            torch.empty(B, Hk, d, dtype=torch.float32, device=dev),
+            torch.empty_like(tv, dtype=torch.uint8) if v8 else None,
+            torch.empty(B, Hk, d, dtype=torch.float32, device=dev) if v8 else None)
+    o = torch.empty_like(tq)
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        sage.sage_smooth_quant_qkv(tq, tk, tv if v8 else None, w.scale, 448.0, out=outs)
+        if evs:
+            evs[1].record(stream)
+        qh, kh, dq, dk, _, vh, dv = outs
+        sage.sage_attn_fwd_quantized(qh, kh, dq, dk, vh if v8 else tv, dv, causal=w.causal,
+                                     variant=variant, o=o)
+        if evs:
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, word = sage.sage_get_device_error()
+    assert st == 0, f"device error {word:#x}"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t_start.record(stream)
+        for s in range(args.steps):
+            # keep the host a few steps ahead, never so far that the launch
+            # queue fills and the GPU waits for the host inside a step
+            if s >= 4:
+                evs[s - 4][2].synchronize()
+            step(evs[s])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    st, word = sage.sage_get_device_error()
+    assert st == 0, f"device error {word:#x}"
+
+    total_ms = t_start.elapsed_time(t_end)
+    attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    t = torch.tensor([total_ms, statistics.mean(attn_ms), statistics.mean(pre_ms)],
+                     dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, attn_avg, pre_avg = (float(x) for x in t.tolist())
+    ms_per_step = total_ms / args.steps
+    value = world * w.ops / (ms_per_step * 1e-3) / 1e12
+
+    # end to end through the public one-call API on pinned host buffers
+    hq, hk, hv = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
+    ho = torch.empty(hq.shape, dtype=torch.float16).pin_memory()
+    sage.sage_attn_fwd_host(hq, hk, hv, ho, causal=w.causal, sm_scale=w.scale, variant=variant)
+    e2e_ms = []
+    for _ in range(args.e2e_steps):
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        sage.sage_attn_fwd_host(hq, hk, hv, ho, causal=w.causal, sm_scale=w.scale,
+                                variant=variant)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+    te = torch.tensor([statistics.mean(e2e_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * w.ops / (float(te.item()) * 1e-3) / 1e12
+    h2d = (q.nbytes + k.nbytes + v.nbytes)
+    d2h = q.nbytes
+
+    peaks = _peaks()
+    if peaks:
+        peak = NOMINAL_8BIT_OVER_BF16 * peaks["bf16_tflops_sustained"]
+        peak_note = ("of measured: MEASURED_PEAKS bf16_tflops_sustained x 2 "
+                     "(nominal 8-bit/bf16 dense ratio)")
+    else:
+        peak = NOMINAL_8BIT_OVER_BF16 * 1400.0
+        peak_note = "of fallback: 1.4 PFLOP/s sustained bf16 x 2"
+    achieved = w.ops / (attn_avg * 1e-3) / 1e12
+    traffic = NCU_TRAFFIC.get((_src_hash(), w.name, variant))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        smp = OracleSampler(w, variant)
+        ops_s, desc = smp.sample(args.ref_budget)
+        cpu = {"value": ops_s / 1e12, "unit": "TOPS", "cores": smp.threads, "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        clocks = clk.summary()
+        prepass_bytes = (q.nbytes * 1.5 + k.nbytes * 2.5 + (v.nbytes * 2.5 if v8 else 0))
+        line = {
+            "metric": "quantized attention TOPS (4BHN^2d/t) at N=32K d=128; % of B200 INT8/FP8 tensor peak",
+            "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8 QK^T + e4m3 PV" if v8 else "int8 QK^T + fp16 PV",
+            "data": "synthetic (seeded numpy, workload recipe; no dataset)",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N,
+                       "d": w.d, "causal": w.causal, "variant": variant,
+                       "global_batch": w.B * world, "seq_len": w.N,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs exceed L2 (Q,K,V %.0f MB > 126 MB); no flush"
+                             % ((q.nbytes + k.nbytes + v.nbytes) / 1e6)},
+            "pct_of_spec_8bit_peak": 100.0 * value / world / SPEC_8BIT_TOPS,
+            "roofline": {"bound": "tensor", "kernel": "attention (k_attn)",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic, "peak_note": peak_note,
+                         "ops_per_launch": w.ops, "avg_launch_ms": attn_avg},
+            "prepass": {"avg_ms": pre_avg, "share": pre_avg / (pre_avg + attn_avg),
+                        "algorithmic_bytes": prepass_bytes,
+                        "gbs": prepass_bytes / (pre_avg * 1e-3) / 1e9},
+            "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": float(te.item())},
+            "gpu_launches": 4 * args.steps,
+            "clocks": {k_: clocks[k_] for k_ in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -95,6 +95,19 @@ sage_status_t sage_quant_v_fp8(const void* v, int B, int H_kv, int N, int d, flo
                                uint8_t* v_hat, float* delta_v, void* stream);
 
 /*
+ * The whole pre-pass in three launches (column statistics of K and V, their
+ * finalisation, one quantization launch for Q, K and V): the results of
+ * sage_smooth_quant_qk and, when v != NULL, of sage_quant_v_fp8 with the
+ * given v_r, bit for bit.  v, v_hat and delta_v are either all NULL
+ * (SAGEAttn-B needs no V pre-pass) or all set.
+ * Scratch: ceil(N/256)*B*H_kv*d*12 bytes, stream-ordered as above.
+ */
+sage_status_t sage_smooth_quant_qkv(const void* q, const void* k, const void* v, int B, int H,
+                                    int H_kv, int N, int d, float sm_scale, float v_r,
+                                    int8_t* q_hat, int8_t* k_hat, uint8_t* v_hat, float* delta_q,
+                                    float* delta_k, float* mean_k, float* delta_v, void* stream);
+
+/*
  * Attention on pre-quantized operands ([SA1] Algorithm 1 steps 3-9, Eq. 4-5):
  * per 128-row q block and ascending 128-key kv tiles,
  *   S = int32(q_hat k_hat^T) * delta_q[i] * delta_k[j]   (tcgen05 kind::i8)

@@ -43,7 +43,7 @@ from typing import Optional, Sequence
 
 import numpy as np
 
-from .codecs import e4m3_decode, e4m3_encode, fp16_rne, FP16_MAX
+from .codecs import e4m3_decode, e4m3_encode, e4m3_round, fp16_rne, FP16_MAX
 
 BLOCK = 128
 F32 = np.float32
@@ -177,7 +177,8 @@ def attention_online(qh, kh, dq, dk, vop, *, causal: bool, operand: str,
                      p_r: float = 448.0, dv=None,
                      q_blocks: Optional[Sequence[int]] = None,
                      s_fp32: bool = True, simulate_f16acc: bool = False,
-                     return_stats: bool = False, out_fp16: bool = True):
+                     return_stats: bool = False, out_fp16: bool = True,
+                     ambiguity: float = 0.0, flip_ambiguous: bool = False):
     """Tiled attention with online softmax, following [SA1] Algorithm 1
     steps 3-9 and Eq. 4-5.
 
@@ -194,6 +195,15 @@ def attention_online(qh, kh, dq, dk, vop, *, causal: bool, operand: str,
     s_fp32: S = fp32(acc) * fp32(dq*dk) as in the kernel; False keeps fp64.
     simulate_f16acc: round every per-tile partial P_hat V_hat to fp16
     (the FP16 accumulator of [SA2++], flushed per tile).
+    ambiguity: relative band eps.  The operand code of an fp32 P~ is
+    decided by floating point; an implementation whose P~ differs from this
+    one by at most a factor (1 +- eps) may legitimately pick the neighbouring
+    code when P~ (times P_r) lies within that band of a rounding midpoint.
+    For every such ambiguous element the difference between the two codes,
+    times |V operand|, is accumulated (with the same online rescaling as O)
+    into a per-output slack; the function then also returns that slack,
+    scaled like O.  flip_ambiguous: use the other code for every ambiguous
+    element (checks that the slack bounds the effect).
     Each q block walks its kv tiles in ascending order; with causal only
     tiles j <= i, masking keys t > r on the diagonal tile."""
     B, H, N, d = qh.shape
@@ -202,6 +212,7 @@ def attention_online(qh, kh, dq, dk, vop, *, causal: bool, operand: str,
     rows = _rows_from_blocks(N, q_blocks)
     rblk = rows // BLOCK
     out = np.zeros((B, H, len(rows), d), dtype=np.float64)
+    slack = np.zeros((B, H, len(rows), d), dtype=np.float64)
     stats = []
     f16acc_overflow = False
     for b in range(B):
@@ -213,6 +224,7 @@ def attention_online(qh, kh, dq, dk, vop, *, causal: bool, operand: str,
             m = np.full(len(rows), -np.inf, dtype=F32 if s_fp32 else np.float64)
             l = np.zeros(len(rows), dtype=np.float64)
             O = np.zeros((len(rows), d), dtype=np.float64)
+            SL = np.zeros((len(rows), d), dtype=np.float64)
             for j in range(nkv):
                 act = (rblk >= j) if causal else np.ones(len(rows), bool)
                 if not act.any():
@@ -242,12 +254,25 @@ def attention_online(qh, kh, dq, dk, vop, *, causal: bool, operand: str,
                 l[ia] = alpha * l[ia] + P.astype(np.float64).sum(axis=1)
                 if operand == "fp16":
                     pop = fp16_rne(P.astype(F32)).astype(np.float64)
+                    rnd = lambda z: fp16_rne(z).astype(np.float64)  # noqa: E731
+                    zv = P.astype(np.float64)
                 elif operand == "e4m3":
                     pop = e4m3_decode(e4m3_encode((P.astype(F32) * F32(p_r)).astype(F32)))
+                    rnd = e4m3_round
+                    zv = P.astype(np.float64) * float(p_r)
                 elif operand == "exact":
                     pop = P.astype(np.float64)
+                    rnd, zv = None, None
                 else:
                     raise ValueError(operand)
+                if ambiguity > 0 and rnd is not None:
+                    lo = rnd(zv * (1.0 - ambiguity))
+                    hi = rnd(zv * (1.0 + ambiguity))
+                    amb = lo != hi
+                    dp = np.where(amb, hi - lo, 0.0)
+                    if flip_ambiguous:
+                        pop = np.where(amb, np.where(pop == lo, hi, lo), pop)
+                    SL[ia] = alpha[:, None] * SL[ia] + dp @ np.abs(Vf[cols])
                 part = pop @ Vf[cols]
                 if simulate_f16acc:
                     if np.abs(part).max(initial=0.0) > FP16_MAX:
@@ -256,21 +281,23 @@ def attention_online(qh, kh, dq, dk, vop, *, causal: bool, operand: str,
                 O[ia] = alpha[:, None] * O[ia] + part
                 m[ia] = m_new
             if operand == "e4m3":
-                res = O * dv[b, hk][None, :].astype(np.float64) / (float(p_r) * l[:, None])
+                scale = dv[b, hk][None, :].astype(np.float64) / (float(p_r) * l[:, None])
             else:
-                res = O / l[:, None]
-            out[b, h] = res
+                scale = 1.0 / l[:, None]
+            out[b, h] = O * scale
+            slack[b, h] = SL * scale
     if out_fp16:
         out = fp16_rne(out)
-    if return_stats or simulate_f16acc:
-        return out, {"tiles": stats, "f16acc_overflow": f16acc_overflow}
+    if return_stats or simulate_f16acc or ambiguity > 0:
+        return out, {"tiles": stats, "f16acc_overflow": f16acc_overflow, "slack": slack}
     return out
 
 
 def sage_attention(q, k, v, *, causal: bool, sm_scale: Optional[float] = None,
                    variant: str = "B", v_r: float = 448.0, p_r: float = 448.0,
                    q_blocks: Optional[Sequence[int]] = None,
-                   simulate_f16acc: bool = False):
+                   simulate_f16acc: bool = False, ambiguity: float = 0.0,
+                   flip_ambiguous: bool = False):
     """Quantized mirror (mode QO) of the whole forward pass: Smooth K,
     per-block INT8 Q/K, then Algorithm 1 with the fp16 (variant "B") or
     E4M3 (variant "8+8") P~V.  Returns (O fp16 [B,H,rows,d], intermediates)."""
@@ -280,20 +307,21 @@ def sage_attention(q, k, v, *, causal: bool, sm_scale: Optional[float] = None,
     qh, dq = quant_q(q, sm_scale)
     kh, dk, mk = smooth_quant_k(k)
     inter = {"q_hat": qh, "delta_q": dq, "k_hat": kh, "delta_k": dk, "mean_k": mk}
+    extra = dict(q_blocks=q_blocks, ambiguity=ambiguity, flip_ambiguous=flip_ambiguous)
     if variant == "B":
-        o = attention_online(qh, kh, dq, dk, v, causal=causal, operand="fp16",
-                             q_blocks=q_blocks)
+        o = attention_online(qh, kh, dq, dk, v, causal=causal, operand="fp16", **extra)
     elif variant == "8+8":
         vh, dv = quant_v_fp8(v, v_r)
         inter.update(v_hat=vh, delta_v=dv)
         o = attention_online(qh, kh, dq, dk, e4m3_decode(vh), causal=causal,
-                             operand="e4m3", p_r=p_r, dv=dv, q_blocks=q_blocks,
-                             simulate_f16acc=simulate_f16acc)
-        if simulate_f16acc:
-            o, st = o
-            inter["f16acc_overflow"] = st["f16acc_overflow"]
+                             operand="e4m3", p_r=p_r, dv=dv,
+                             simulate_f16acc=simulate_f16acc, **extra)
     else:
         raise ValueError(variant)
+    if isinstance(o, tuple):
+        o, st = o
+        inter["f16acc_overflow"] = st["f16acc_overflow"]
+        inter["slack"] = st["slack"]
     return o, inter
 
 

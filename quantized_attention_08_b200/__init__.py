@@ -6,7 +6,8 @@ memory and the current stream.  There is no fallback: if the library is not
 built, or the GPU is not a B200, the calls raise.
 
 Functions carry the names of the C entry points:
-  sage_smooth_quant_qk, sage_quant_v_fp8, sage_attn_fwd_quantized,
+  sage_smooth_quant_qk, sage_quant_v_fp8, sage_smooth_quant_qkv,
+  sage_attn_fwd_quantized,
   sage_attn_fwd, sage_attn_fwd_ws, sage_attn_workspace_bytes,
   sage_attn_fwd_host, sage_get_device_error, sage_set_wait_timeout_ns,
   sage_selftest_wait_timeout, sage_status_string, sage_version,
@@ -36,6 +37,8 @@ _f = _c.c_float
 _SIGS = {
     "sage_smooth_quant_qk": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp]),
     "sage_quant_v_fp8": (_i, [_vp, _i, _i, _i, _i, _f, _vp, _vp, _vp]),
+    "sage_smooth_quant_qkv": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp, _vp,
+                                   _vp, _vp, _vp, _vp]),
     "sage_attn_fwd_quantized": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "sage_attn_workspace_bytes": (_c.c_size_t, [_i, _i, _i, _i, _i, _i]),
     "sage_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
@@ -161,6 +164,34 @@ def sage_quant_v_fp8(v: torch.Tensor, v_r: float = 448.0, out=None, stream=None)
     st = load_library().sage_quant_v_fp8(_ptr(v), B, Hk, N, d, float(v_r), _ptr(vh), _ptr(dv),
                                          _stream(stream))
     _check(st, "sage_quant_v_fp8")
+    return out
+
+
+def sage_smooth_quant_qkv(q, k, v=None, sm_scale: Optional[float] = None, v_r: float = 448.0,
+                          out=None, stream=None):
+    """Whole pre-pass in three launches.  Returns (q_hat, k_hat, delta_q,
+    delta_k, mean_k, v_hat, delta_v); the last two are None when v is None."""
+    _need(q, torch.float16, "q")
+    _need(k, torch.float16, "k")
+    if v is not None:
+        _need(v, torch.float16, "v")
+    B, H, N, d = q.shape
+    Hk = k.shape[1]
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        dev = q.device
+        out = (torch.empty_like(q, dtype=torch.int8), torch.empty_like(k, dtype=torch.int8),
+               torch.empty(B, H, _nb(N), dtype=torch.float32, device=dev),
+               torch.empty(B, Hk, _nb(N), dtype=torch.float32, device=dev),
+               torch.empty(B, Hk, d, dtype=torch.float32, device=dev),
+               None if v is None else torch.empty_like(v, dtype=torch.uint8),
+               None if v is None else torch.empty(B, Hk, d, dtype=torch.float32, device=dev))
+    qh, kh, dq, dk, mk, vh, dv = out
+    st = load_library().sage_smooth_quant_qkv(
+        _ptr(q), _ptr(k), _ptr(v), B, H, Hk, N, d, float(sm_scale), float(v_r), _ptr(qh),
+        _ptr(kh), _ptr(vh), _ptr(dq), _ptr(dk), _ptr(mk), _ptr(dv), _stream(stream))
+    _check(st, "sage_smooth_quant_qkv")
     return out
 
 

@@ -9,15 +9,24 @@
 //       static delta_P = 1/448 and per-channel delta_V.
 //
 // One CTA owns two 128-row q tiles of one (batch, head) and streams the kv
-// tiles of that head through a multi-stage TMA/mbarrier ring:
-//   warp 8      TMA producer (Q once, then K_j and V_j per stage)
-//   warp 9      MMA issuer: S_g = Q_g K_j^T (kind::i8 -> s32 in TMEM),
-//               O_g += P_g V_j (kind::f16 or kind::f8f6f4, P_g read from TMEM)
+// tiles of that head through a multi-stage TMA/mbarrier ring.  16 warps:
 //   warps 0-3   softmax of q tile 0, warps 4-7 softmax of q tile 1: each
-//               thread owns one row; it reads S from TMEM, keeps m and l in
-//               registers, writes P~ (fp16, or e4m3 of 448 P~) back into the
-//               TMEM columns of S, rescales its row of O when m moves, and
-//               finally normalises O and stores fp16.
+//               thread owns one row; it reads S from TMEM, keeps the running
+//               max m and sum l in registers, hands the row's rescale factor
+//               alpha = 2^(m_old - m_new) to the correction warps through
+//               shared memory right after the row max (so the rescale of O
+//               overlaps the exponentials), and writes P~ (fp16, or e4m3 of
+//               448 P~) back into the TMEM columns of S.
+//   warps 8-11  correction: rescale the rows of O_g in TMEM by alpha before
+//               the next P~V accumulates into them, and the epilogue
+//               (O / l, x delta_v[c] / 448 for 8+8, fp16 store).
+//   warp 12     MMA issuer (one thread): S_g = Q_g K_j^T (kind::i8, s32 in
+//               TMEM) and O_g += P_g V_j (kind::f16 / kind::f8f6f4, P_g from TMEM).
+//   warp 13     TMA producer (Q once, then K_j, V_j per ring stage).
+//   warps 14-15 idle (complete the last warpgroup for setmaxnreg).
+// Registers: launched at 128 per thread; the softmax warpgroups grow to 192,
+// the correction warpgroup shrinks to 72 and the last warpgroup to 56
+// (8*192 + 4*72 + 4*56 = 16*128 per lane; per SM sub-partition 192+192+72+56).
 // Tensor memory (512 columns x 128 lanes): S_0 [0,128), S_1 [128,256),
 // O_0 [256,256+d), O_1 [384,384+d); P_g aliases the first columns of S_g.
 // Every wait is bounded (see mbar_wait); on expiry the CTA records the
@@ -32,8 +41,9 @@
 namespace sage {
 
 constexpr int kBM = 128, kBN = 128;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
-constexpr int kAttnThreads = 320;
+constexpr int kMmaWarp = 12, kProducerWarp = 13;  // warps 8-11: correction
+constexpr int kAttnThreads = 512;
+constexpr uint32_t kRegSoftmax = 192, kRegCorr = 72, kRegMisc = 56;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2P448 = 8.807354922057604f;  // log2(448): P operand = 448 * P~
 
@@ -46,8 +56,10 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NS * K_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NS * V_BYTES;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int OFF_BAR = OFF_V + NS * V_BYTES;       // barriers, 512 B
+  static constexpr int OFF_ALPHA = OFF_BAR + 512;            // float [2][128]
+  static constexpr int OFF_L = OFF_ALPHA + 2 * 128 * 4;      // float [2][128]
+  static constexpr int SMEM = OFF_L + 2 * 128 * 4 + 1024;    // + alignment slack
   // Q_hat / K_hat: K-major int8 rows of D bytes, swizzle span = row length.
   static constexpr uint32_t QK_SW = (D == 128) ? SW_128B : SW_64B;
   static constexpr uint32_t QK_SBO = 8 * D;
@@ -85,38 +97,76 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
   }
 }
 
-// Softmax of one 128-column tile for this thread's row.  `a` holds the s32
-// scores on entry and the packed P operand on exit (fp16x2, or 4 x e4m3).
-// c = delta_q * delta_k * log2(e); m is the running max in the log2 domain.
-// Columns >= lim are masked (only when MASKED).  Returns the new max and
-// the row sum of this tile's (unrounded) P values.
-template <int VAR, bool MASKED>
-__device__ __forceinline__ float softmax_tile(uint32_t (&a)[128], float c, float m, int lim,
-                                              float& rowsum) {
+// ---------------------------------------------------------------- packed fp32 pairs
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 up2(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// Row max of the s32 scores of one tile (columns >= lim masked when MASKED):
+// eight independent 3-input chains, then a tree.
+template <bool MASKED>
+__device__ __forceinline__ int tile_rowmax(uint32_t (&a)[128], int lim) {
   if (MASKED) {
 #pragma unroll
     for (int i = 0; i < 128; ++i)
       if (i >= lim) a[i] = 0x80000000u;
   }
-  int imax = static_cast<int>(a[0]);
+  int mx[8];
 #pragma unroll
-  for (int i = 1; i < 128; ++i) imax = max(imax, static_cast<int>(a[i]));
-  // |imax| <= d * 127^2 < 2^22: the int -> float conversion is exact.
-  const float m_new = fmaxf(m, __fmul_rn(static_cast<float>(imax), c));
-  const float bias = (VAR == 1) ? (kLog2P448 - m_new) : -m_new;
-  float s0 = 0.f, s1 = 0.f;
+  for (int t = 0; t < 8; ++t) {
+    mx[t] = __vimax3_s32(static_cast<int>(a[16 * t]), static_cast<int>(a[16 * t + 1]),
+                         static_cast<int>(a[16 * t + 2]));
+#pragma unroll
+    for (int i = 3; i < 15; i += 2)
+      mx[t] = __vimax3_s32(mx[t], static_cast<int>(a[16 * t + i]), static_cast<int>(a[16 * t + i + 1]));
+    mx[t] = max(mx[t], static_cast<int>(a[16 * t + 15]));
+  }
+  return max(__vimax3_s32(mx[0], mx[1], mx[2]), max(__vimax3_s32(mx[3], mx[4], mx[5]), max(mx[6], mx[7])));
+}
+// P~ of one tile for this thread's row: p = 2^(acc*c + bias) with
+// c = delta_q * delta_k * log2(e), bias = -m_new (+ log2 448 for 8+8).  `a`
+// holds the s32 scores on entry and the packed P operand on exit (fp16x2, or
+// 4 x e4m3 per word; lower columns in lower bits).  Returns the row sum of
+// the unrounded P values.
+template <int VAR, bool MASKED>
+__device__ __forceinline__ float tile_exp(uint32_t (&a)[128], float c, float bias, int lim) {
+  const uint64_t c2 = pk2(c, c), b2 = pk2(bias, bias), magic2 = pk2(-12582912.f, -12582912.f);
+  uint64_t sum2[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) sum2[t] = 0;
 #pragma unroll
   for (int i = 0; i < 128; i += 4) {
     float p[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      // exact int -> float: 1.5*2^23 + a has unit spacing for |a| < 2^22
-      const float f = __fsub_rn(__uint_as_float(a[i + e] + 0x4B400000u), 12582912.f);
-      p[e] = ex2_approx(__fmaf_rn(f, c, bias));
-      if (MASKED && i + e >= lim) p[e] = 0.f;
+    for (int e = 0; e < 4; e += 2) {
+      const uint64_t f2 = add2(pk2(__uint_as_float(a[i + e] + 0x4B400000u),
+                                   __uint_as_float(a[i + e + 1] + 0x4B400000u)), magic2);
+      const float2 x = up2(fma2(f2, c2, b2));
+      p[e] = ex2_approx(x.x);
+      p[e + 1] = ex2_approx(x.y);
+      if (MASKED) {
+        if (i + e >= lim) p[e] = 0.f;
+        if (i + e + 1 >= lim) p[e + 1] = 0.f;
+      }
     }
-    s0 += p[0] + p[1];
-    s1 += p[2] + p[3];
+    sum2[(i / 4) & 3] = add2(sum2[(i / 4) & 3], add2(pk2(p[0], p[1]), pk2(p[2], p[3])));
     if (VAR == 0) {
       a[i / 2] = pack_f16x2(p[0], p[1]);
       a[i / 2 + 1] = pack_f16x2(p[2], p[3]);
@@ -124,12 +174,11 @@ __device__ __forceinline__ float softmax_tile(uint32_t (&a)[128], float c, float
       a[i / 4] = pack_e4m3x2(p[0], p[1]) | (pack_e4m3x2(p[2], p[3]) << 16);
     }
   }
-  rowsum = s0 + s1;
-  return m_new;
+  const float2 s = up2(add2(add2(sum2[0], sum2[1]), add2(sum2[2], sum2[3])));
+  return s.x + s.y;
 }
 
 template <int D, int VAR, bool CAUSAL>
-// 10 warps: up to 3 share one SM sub-partition's 16K registers -> <= 168 per thread.
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, const AttnKParams p) {
@@ -141,16 +190,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sK = smem + C::OFF_K;
   uint8_t* sV = smem + C::OFF_V;
+  float* s_alpha = reinterpret_cast<float*>(smem + C::OFF_ALPHA);  // [2][128]
+  float* s_l = reinterpret_cast<float*>(smem + C::OFF_L);          // [2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* bar_q = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* k_empty = k_full + NS;
   uint64_t* v_full = k_empty + NS;
   uint64_t* v_empty = v_full + NS;
-  uint64_t* s_full = v_empty + NS;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 2;
-  uint64_t* mma_done = pv_done + 2;
+  uint64_t* s_full = v_empty + NS;   // [2] S_g(j) in TMEM          (MMA commit)
+  uint64_t* p_full = s_full + 2;     // [2] P_g(j) in TMEM          (128 softmax threads)
+  uint64_t* a_full = p_full + 2;     // [2] alpha_g(j) in smem      (128 softmax threads)
+  uint64_t* o_ready = a_full + 2;    // [2] O_g rescaled for j      (128 correction threads)
+  uint64_t* pv_done = o_ready + 2;   // [2] PV_g(j) complete        (MMA commit)
+  uint64_t* l_full = pv_done + 2;    // [2] final l_g in smem       (128 softmax threads)
+  uint64_t* mma_done = l_full + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
@@ -179,7 +233,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int g = 0; g < 2; ++g) {
       mbar_init(&s_full[g], 1);
       mbar_init(&p_full[g], 128);
+      mbar_init(&a_full[g], 128);
+      mbar_init(&o_ready[g], 128);
       mbar_init(&pv_done[g], 1);
+      mbar_init(&l_full[g], 128);
     }
     mbar_init(mma_done, 1);
     *s_abort = 0;
@@ -194,8 +251,202 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
 
-  if (warp == kProducerWarp) {
-    if (lane == 0) {
+  if (warp < 8) {
+    // ---------------------------------------------------------------- softmax
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax));
+    const int g = warp >> 2, wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const int qb = qb0 + g;
+    if (g == 0 || has1) {
+      const int nkv_g = g == 0 ? nkv0 : nkv1;
+      const uint32_t tS = tmem + (static_cast<uint32_t>(wq * 32) << 16) + g * 128;
+      const float dq_l2e = __fmul_rn(p.dq[static_cast<size_t>(bh) * p.nqb + qb], kLog2e);
+      const float* dkp = p.dk + static_cast<size_t>(zkv) * p.nkvb;
+      float m = -INFINITY, l = 0.f;
+      float dk_next = dkp[0];
+      for (int j = 0; j < nkv_g; ++j) {
+        const float c = __fmul_rn(dq_l2e, dk_next);
+        if (j + 1 < nkv_g) dk_next = dkp[j + 1];
+        // tcgen05.ld/st below are warp-collective: every lane takes the same branch
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[g], j & 1, s_abort, tlim, 8))) break;
+        tc_fence_after();
+        uint32_t a[128];
+        SAGE_TMEM_LD32(tS + 0, a);
+        SAGE_TMEM_LD32(tS + 32, (a + 32));
+        SAGE_TMEM_LD32(tS + 64, (a + 64));
+        SAGE_TMEM_LD32(tS + 96, (a + 96));
+        tmem_wait_ld();
+        const int valid = p.N - j * kBN;  // keys left in this tile
+        const bool masked = (CAUSAL && j == qb) || valid < kBN;
+        const int lim = masked ? min(valid, (CAUSAL && j == qb) ? r + 1 : kBN) : kBN;
+        const int imax = masked ? tile_rowmax<true>(a, lim) : tile_rowmax<false>(a, lim);
+        // |imax| <= d * 127^2 < 2^22: the int -> float conversion is exact.
+        const float m_new = fmaxf(m, __fmul_rn(static_cast<float>(imax), c));
+        const float alpha = ex2_approx(m - m_new);  // 0 on the first tile
+        if (j > 0) {
+          // the correction warps rescale O_g while this thread computes P~
+          s_alpha[g * 128 + r] = alpha;
+          mbar_arrive(&a_full[g]);
+        }
+        const float bias = (VAR == 1) ? (kLog2P448 - m_new) : -m_new;
+        const float rs = masked ? tile_exp<VAR, true>(a, c, bias, lim) : tile_exp<VAR, false>(a, c, bias, lim);
+        if (VAR == 0) {
+          SAGE_TMEM_ST32(tS + 0, a);
+          SAGE_TMEM_ST32(tS + 32, (a + 32));
+        } else {
+          SAGE_TMEM_ST32(tS + 0, a);
+        }
+        l = __fmaf_rn(alpha, l, rs);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[g]);
+        m = m_new;
+      }
+      s_l[g * 128 + r] = l;
+      mbar_arrive(&l_full[g]);
+    }
+  } else if (warp < 12) {
+    // ---------------------------------------------------------------- correction + epilogue
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegCorr));
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    bool ok = true;
+    // rescale of O_g for step j (j >= 1), in the order the MMA issuer consumes them
+    for (int j = 1; ok && j < nkv; ++j) {
+      for (int g = 0; g < 2; ++g) {
+        if (g == 0 ? (j >= nkv0) : (!has1 || j >= nkv1)) continue;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&a_full[g], (j - 1) & 1, s_abort, tlim, 10))) {
+          ok = false;
+          break;
+        }
+        const float alpha = s_alpha[g * 128 + r];
+        // O_g holds PV_g(j-1), complete: the softmax saw S_g(j), whose commit
+        // covered every earlier MMA.
+        if (__any_sync(0xFFFFFFFFu, alpha != 1.f)) {
+          tc_fence_after();
+          const uint32_t tO = tmem + lane_off + 256 + g * 128;
+#pragma unroll 1
+          for (int cb = 0; cb < D / 32; ++cb) {
+            uint32_t o[32];
+            SAGE_TMEM_LD32(tO + cb * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            SAGE_TMEM_ST32(tO + cb * 32, o);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(&o_ready[g]);
+      }
+    }
+    // epilogue: O / l (x delta_v[c] / 448 for 8+8, folded into l), fp16 rows
+    for (int g = 0; ok && g < 2; ++g) {
+      if (g == 1 && !has1) break;
+      const int nkv_g = g == 0 ? nkv0 : nkv1;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&l_full[g], 0, s_abort, tlim, 11) &&
+                                       mbar_wait(&pv_done[g], (nkv_g - 1) & 1, s_abort, tlim, 9)))
+        break;
+      tc_fence_after();
+      const float inv = 1.f / s_l[g * 128 + r];
+      const int row = (qb0 + g) * kBM + r;
+      const uint32_t tO = tmem + lane_off + 256 + g * 128;
+      uint4* orow = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * p.N + row) * D);
+      const float* dvp = p.dv + static_cast<size_t>(zkv) * D;
+#pragma unroll 1
+      for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t o[32];
+        SAGE_TMEM_LD32(tO + cb * 32, o);
+        tmem_wait_ld();
+        uint32_t hv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float x0 = __uint_as_float(o[2 * i]) * inv;
+          float x1 = __uint_as_float(o[2 * i + 1]) * inv;
+          if (VAR == 1) {
+            x0 *= dvp[cb * 32 + 2 * i];
+            x1 *= dvp[cb * 32 + 2 * i + 1];
+          }
+          hv[i] = pack_f16x2(x0, x1);
+        }
+        if (row < p.N) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            orow[cb * 4 + i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+        }
+      }
+    }
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegMisc));
+    if (warp == kMmaWarp && lane == 0) {
+      // Issue order per kv step i (two q tiles ping-pong on the tensor core):
+      //   S_0(i), PV_1(i-1), S_1(i), PV_0(i)
+      // so softmax 0 of step i overlaps PV_1(i-1) + S_1(i) and softmax 1
+      // overlaps PV_0(i) + S_0(i+1).  S_g(i+1) overwrites the TMEM columns
+      // that PV_g(i) reads P_g from; tcgen05.mma ops issued by one thread
+      // execute in order, so the read precedes the overwrite.  The commit
+      // after S_g(i+1) therefore also certifies that PV_g(i) completed, which
+      // is what lets the correction warps rescale O_g once S_g(i+1) is seen.
+      const uint64_t dQ0 = sdesc(smem_u32(sQ), 16, C::QK_SBO, C::QK_SW);
+      const uint64_t dK0 = sdesc(smem_u32(sK), 16, C::QK_SBO, C::QK_SW);
+      const uint64_t dV0 = sdesc(smem_u32(sV), C::V_LBO, C::V_SBO, C::V_SW);
+      int k_seen = -1, v_seen = -1;
+      auto active = [&](int g, int j) { return g == 0 ? (j < nkv0) : (has1 && j < nkv1); };
+      auto issue_s = [&](int g, int j) -> bool {
+        if (!active(g, j)) return true;
+        if (k_seen < j) {
+          if (!mbar_wait(&k_full[j % NS], (j / NS) & 1, s_abort, tlim, 4)) return false;
+          k_seen = j;
+        }
+        tc_fence_after();
+        const uint64_t ad = dQ0 + (g * C::Q_BYTES >> 4);
+        const uint64_t bd = dK0 + ((j % NS) * C::K_BYTES >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk)
+          mma_i8_ss(tmem + g * 128, ad + kk * 2, bd + kk * 2, C::IDESC_QK, kk > 0 ? 1u : 0u);
+        tc_commit(&s_full[g]);
+        return true;
+      };
+      auto issue_pv = [&](int g, int j) -> bool {
+        if (!active(g, j)) return true;
+        if (v_seen < j) {
+          if (!mbar_wait(&v_full[j % NS], (j / NS) & 1, s_abort, tlim, 6)) return false;
+          v_seen = j;
+        }
+        if (!mbar_wait(&p_full[g], j & 1, s_abort, tlim, 7)) return false;
+        if (j > 0 && !mbar_wait(&o_ready[g], (j - 1) & 1, s_abort, tlim, 12)) return false;
+        tc_fence_after();
+        const uint64_t vd = dV0 + ((j % NS) * C::V_BYTES >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kBN / C::PV_K; ++kk) {
+          const uint64_t bd = vd + (kk * C::PV_K * C::V_ROW >> 4);
+          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+          if (VAR == 0)
+            mma_f16_ts(tmem + 256 + g * 128, tmem + g * 128 + kk * 8, bd, C::IDESC_PV, acc);
+          else
+            mma_f8_ts(tmem + 256 + g * 128, tmem + g * 128 + kk * 8, bd, C::IDESC_PV, acc);
+        }
+        tc_commit(&pv_done[g]);
+        return true;
+      };
+      bool ok = mbar_wait(bar_q, 0, s_abort, tlim, 3);
+      ok = ok && issue_s(0, 0) && issue_s(1, 0);
+      if (ok) tc_commit(&k_empty[0]);
+      ok = ok && issue_pv(0, 0);
+      for (int i = 1; ok && i < nkv; ++i) {
+        ok = issue_s(0, i) && issue_pv(1, i - 1);
+        if (!ok) break;
+        tc_commit(&v_empty[(i - 1) % NS]);
+        ok = issue_s(1, i);
+        if (!ok) break;
+        tc_commit(&k_empty[i % NS]);
+        ok = issue_pv(0, i);
+      }
+      if (ok && issue_pv(1, nkv - 1)) tc_commit(&v_empty[(nkv - 1) % NS]);
+      tc_commit(mma_done);
+      drain_wait(mma_done, 0, tlim);
+    } else if (warp == kProducerWarp && lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -225,152 +476,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         drain_wait(bar_q, 0, tlim);
         for (int i = max(0, nk - NS); i < nk; ++i) drain_wait(&k_full[i % NS], (i / NS) & 1, tlim);
         for (int i = max(0, nv - NS); i < nv; ++i) drain_wait(&v_full[i % NS], (i / NS) & 1, tlim);
-      }
-    }
-  } else if (warp == kMmaWarp) {
-    if (lane == 0) {
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      bool ok = mbar_wait(bar_q, 0, s_abort, tlim, 3);
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % NS;
-        const uint32_t ph = (j / NS) & 1;
-        if (!mbar_wait(&k_full[s], ph, s_abort, tlim, 4)) break;
-        for (int g = 0; g < 2 && ok; ++g) {
-          if (g == 1 ? !has1 : (j >= nkv0)) continue;
-          // S_g (aliasing P_g) may be overwritten once PV_g(j-1) has read P_g
-          if (j > 0 && !mbar_wait(&pv_done[g], (j - 1) & 1, s_abort, tlim, 5)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk) {
-            const uint64_t ad = sdesc(aQ + g * C::Q_BYTES + kk * 32, 16, C::QK_SBO, C::QK_SW);
-            const uint64_t bd = sdesc(aK + s * C::K_BYTES + kk * 32, 16, C::QK_SBO, C::QK_SW);
-            mma_i8_ss(tmem + g * 128, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&s_full[g]);
-        }
-        if (!ok) break;
-        tc_commit(&k_empty[s]);
-        if (!mbar_wait(&v_full[s], ph, s_abort, tlim, 6)) break;
-        for (int g = 0; g < 2 && ok; ++g) {
-          if (g == 1 ? !has1 : (j >= nkv0)) continue;
-          if (!mbar_wait(&p_full[g], j & 1, s_abort, tlim, 7)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kBN / C::PV_K; ++kk) {
-            const uint64_t bd = sdesc(aV + s * C::V_BYTES + kk * C::PV_K * C::V_ROW, C::V_LBO,
-                                      C::V_SBO, C::V_SW);
-            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-            if (VAR == 0)
-              mma_f16_ts(tmem + 256 + g * 128, tmem + g * 128 + kk * 8, bd, C::IDESC_PV, acc);
-            else
-              mma_f8_ts(tmem + 256 + g * 128, tmem + g * 128 + kk * 8, bd, C::IDESC_PV, acc);
-          }
-          tc_commit(&pv_done[g]);
-        }
-        if (!ok) break;
-        tc_commit(&v_empty[s]);
-      }
-      tc_commit(mma_done);
-      drain_wait(mma_done, 0, tlim);
-    }
-  } else {
-    // ---------------------------------------------------------------- softmax
-    const int g = warp >> 2, wq = warp & 3;
-    const int r = wq * 32 + lane;
-    const int qb = qb0 + g;
-    if (g == 0 || has1) {
-      const int nkv_g = g == 0 ? nkv0 : nkv1;
-      const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-      const uint32_t tS = tmem + lane_off + g * 128;
-      const uint32_t tO = tmem + lane_off + 256 + g * 128;
-      const float dq_l2e = __fmul_rn(p.dq[static_cast<size_t>(bh) * p.nqb + qb], kLog2e);
-      const float* dkp = p.dk + static_cast<size_t>(zkv) * p.nkvb;
-      float m = -INFINITY, l = 0.f;
-      bool ok = true;
-      float dk_next = dkp[0];
-      for (int j = 0; j < nkv_g; ++j) {
-        const float c = __fmul_rn(dq_l2e, dk_next);
-        if (j + 1 < nkv_g) dk_next = dkp[j + 1];
-        // tcgen05.ld/st below are warp-collective: every lane takes the same branch
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[g], j & 1, s_abort, tlim, 8))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        uint32_t a[128];
-        SAGE_TMEM_LD32(tS + 0, a);
-        SAGE_TMEM_LD32(tS + 32, (a + 32));
-        SAGE_TMEM_LD32(tS + 64, (a + 64));
-        SAGE_TMEM_LD32(tS + 96, (a + 96));
-        tmem_wait_ld();
-        const int valid = p.N - j * kBN;  // keys left in this tile
-        const bool masked = (CAUSAL && j == qb) || valid < kBN;
-        float rs, m_new;
-        if (masked) {
-          const int lim = min(valid, (CAUSAL && j == qb) ? r + 1 : kBN);
-          m_new = softmax_tile<VAR, true>(a, c, m, lim, rs);
-        } else {
-          m_new = softmax_tile<VAR, false>(a, c, m, kBN, rs);
-        }
-        if (VAR == 0) {
-          SAGE_TMEM_ST32(tS + 0, a);
-          SAGE_TMEM_ST32(tS + 32, (a + 32));
-        } else {
-          SAGE_TMEM_ST32(tS + 0, a);
-        }
-        const float alpha = ex2_approx(m - m_new);  // 0 on the first tile
-        l = __fmaf_rn(alpha, l, rs);
-        if (j > 0 && __any_sync(0xFFFFFFFFu, m_new > m)) {
-          // O_g holds PV_g(j-1), complete: S_g(j) was issued after it.
-#pragma unroll 1
-          for (int cb = 0; cb < D / 32; ++cb) {
-            uint32_t o[32];
-            SAGE_TMEM_LD32(tO + cb * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            SAGE_TMEM_ST32(tO + cb * 32, o);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&p_full[g]);
-        m = m_new;
-      }
-      if (ok && __all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[g], (nkv_g - 1) & 1, s_abort, tlim, 9))) {
-        tc_fence_after();
-        const float inv = 1.f / l;
-        const int row = qb * kBM + r;
-        uint4* orow = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * p.N + row) * D);
-        const float* dvp = p.dv + static_cast<size_t>(zkv) * D;
-#pragma unroll 1
-        for (int cb = 0; cb < D / 32; ++cb) {
-          uint32_t o[32];
-          SAGE_TMEM_LD32(tO + cb * 32, o);
-          tmem_wait_ld();
-          uint32_t hv[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float x0 = __uint_as_float(o[2 * i]) * inv;
-            float x1 = __uint_as_float(o[2 * i + 1]) * inv;
-            if (VAR == 1) {
-              x0 *= dvp[cb * 32 + 2 * i];
-              x1 *= dvp[cb * 32 + 2 * i + 1];
-            }
-            hv[i] = pack_f16x2(x0, x1);
-          }
-          if (row < p.N) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              orow[cb * 4 + i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
-          }
-        }
       }
     }
   }

@@ -129,11 +129,13 @@ __global__ void k_finalize(const long long* __restrict__ ksum, const uint32_t* _
 // System/6000 processor", IBM J. Res. Dev. 34(1), 1990): q = RN(x*r) is
 // within one ulp of x/d, the remainder x - q*d is exact in one fma, and
 // RN(q + rem*r) is the correctly rounded quotient.  Valid away from
-// overflow/underflow, which the quantizer's ranges never reach.
+// overflow/underflow, which the quantizer's ranges never reach.  The
+// correction's additions turn a -0 quotient into +0; with d > 0 the quotient
+// carries the sign of x, which copysign restores (E4M3 encodes -0 as 0x80).
 __device__ __forceinline__ float div_rn_by(float x, float d, float r) {
   const float q = __fmul_rn(x, r);
   const float rem = __fmaf_rn(-q, d, x);
-  return __fmaf_rn(rem, r, q);
+  return copysignf(__fmaf_rn(rem, r, q), x);
 }
 
 // Round-half-even of |y| <= 127 to an int8 code: adding 1.5*2^23 leaves the

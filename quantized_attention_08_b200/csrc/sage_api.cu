@@ -4,7 +4,7 @@
 #include <cmath>
 #include <cstring>
 
-#include "../../include/sage.h"
+#include "sage.h"
 #include "sage_internal.h"
 
 namespace {
@@ -78,30 +78,20 @@ WsLayout ws_layout(int B, int H, int H_kv, int N, int d, int variant) {
   return L;
 }
 
-// The whole pass with intermediates carved from `ws` (L.total bytes).
-sage_status_t run_forward(const void* q, const void* k, const void* v, void* o, int B, int H,
-                          int H_kv, int N, int d, int causal, float sm_scale, int variant,
-                          uint8_t* ws, const WsLayout& L, cudaStream_t st) {
-  const bool v8 = variant == SAGE_VARIANT_8P8;
+// Pre-pass for Q, K and (when v != nullptr) V with caller-provided scratch.
+cudaError_t run_prepass(const void* q, const void* k, const void* v, int B, int H, int H_kv, int N,
+                        int d, float sm_scale, float v_r, int8_t* q_hat, int8_t* k_hat,
+                        uint8_t* v_hat, float* delta_q, float* delta_k, float* mean_k,
+                        float* delta_v, long long* ksum, uint32_t* vmax, cudaStream_t st) {
   const int slabs = B * H_kv;
-  int8_t* q_hat = reinterpret_cast<int8_t*>(ws + L.q_hat);
-  int8_t* k_hat = reinterpret_cast<int8_t*>(ws + L.k_hat);
-  uint8_t* v_hat = v8 ? ws + L.v_hat : nullptr;
-  float* delta_q = reinterpret_cast<float*>(ws + L.delta_q);
-  float* delta_k = reinterpret_cast<float*>(ws + L.delta_k);
-  float* mean_k = reinterpret_cast<float*>(ws + L.mean_k);
-  float* delta_v = v8 ? reinterpret_cast<float*>(ws + L.delta_v) : nullptr;
-  long long* ksum = reinterpret_cast<long long*>(ws + L.ksum);
-  uint32_t* vmax = v8 ? reinterpret_cast<uint32_t*>(ws + L.vmax) : nullptr;
-
-  cudaError_t e = sage::launch_colstats(k, v8 ? v : nullptr, slabs, N, d, ksum, vmax, st);
+  cudaError_t e = sage::launch_colstats(k, v, slabs, N, d, ksum, v ? vmax : nullptr, st);
   if (e == cudaSuccess)
-    e = sage::launch_finalize(ksum, vmax, slabs, N, d, 448.0f, mean_k, delta_v, st);
+    e = sage::launch_finalize(ksum, v ? vmax : nullptr, slabs, N, d, v_r, mean_k, delta_v, st);
   if (e == cudaSuccess) {
     sage::QuantArgs qa;
     qa.q = q;
     qa.k = k;
-    qa.v = v8 ? v : nullptr;
+    qa.v = v;
     qa.q_hat = q_hat;
     qa.k_hat = k_hat;
     qa.v_hat = v_hat;
@@ -117,6 +107,26 @@ sage_status_t run_forward(const void* q, const void* k, const void* v, void* o, 
     qa.d = d;
     e = sage::launch_quant(qa, st);
   }
+  return e;
+}
+
+// The whole pass with intermediates carved from `ws` (L.total bytes).
+sage_status_t run_forward(const void* q, const void* k, const void* v, void* o, int B, int H,
+                          int H_kv, int N, int d, int causal, float sm_scale, int variant,
+                          uint8_t* ws, const WsLayout& L, cudaStream_t st) {
+  const bool v8 = variant == SAGE_VARIANT_8P8;
+  int8_t* q_hat = reinterpret_cast<int8_t*>(ws + L.q_hat);
+  int8_t* k_hat = reinterpret_cast<int8_t*>(ws + L.k_hat);
+  uint8_t* v_hat = v8 ? ws + L.v_hat : nullptr;
+  float* delta_q = reinterpret_cast<float*>(ws + L.delta_q);
+  float* delta_k = reinterpret_cast<float*>(ws + L.delta_k);
+  float* mean_k = reinterpret_cast<float*>(ws + L.mean_k);
+  float* delta_v = v8 ? reinterpret_cast<float*>(ws + L.delta_v) : nullptr;
+  long long* ksum = reinterpret_cast<long long*>(ws + L.ksum);
+  uint32_t* vmax = v8 ? reinterpret_cast<uint32_t*>(ws + L.vmax) : nullptr;
+
+  cudaError_t e = run_prepass(q, k, v8 ? v : nullptr, B, H, H_kv, N, d, sm_scale, 448.0f, q_hat,
+                              k_hat, v_hat, delta_q, delta_k, mean_k, delta_v, ksum, vmax, st);
   if (e == cudaSuccess) {
     sage::AttnArgs aa;
     aa.q_hat = q_hat;
@@ -230,6 +240,38 @@ sage_status_t sage_quant_v_fp8(const void* v, int B, int H_kv, int N, int d, flo
     qa.d = d;
     e = sage::launch_quant(qa, st);
   }
+  cudaError_t ef = cudaFreeAsync(scratch, st);
+  return from_cuda(e != cudaSuccess ? e : ef);
+}
+
+sage_status_t sage_smooth_quant_qkv(const void* q, const void* k, const void* v, int B, int H,
+                                    int H_kv, int N, int d, float sm_scale, float v_r,
+                                    int8_t* q_hat, int8_t* k_hat, uint8_t* v_hat, float* delta_q,
+                                    float* delta_k, float* mean_k, float* delta_v, void* stream) {
+  sage_status_t s = check_sizes(B, H, H_kv, N, d);
+  if (s != SAGE_OK) return s;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  const bool hv = v != nullptr;
+  if (hv && (!(v_r > 0.f) || !(v_r <= 448.f))) return SAGE_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return SAGE_OK;
+  if (!q || !k || !q_hat || !k_hat || !delta_q || !delta_k || !mean_k) return SAGE_ERR_INVALID_ARG;
+  if (hv != (v_hat != nullptr) || hv != (delta_v != nullptr)) return SAGE_ERR_INVALID_ARG;
+  if (!a16(q) || !a16(k) || !a16(q_hat) || !a16(k_hat) || !a4(delta_q) || !a4(delta_k) ||
+      !a4(mean_k) || (hv && (!a16(v) || !a16(v_hat) || !a4(delta_v))))
+    return SAGE_ERR_MISALIGNED;
+  if ((s = check_device()) != SAGE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n = static_cast<size_t>(B) * H_kv * sage::stat_chunks(N) * d;
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocAsync(&scratch, n * 12, st);
+  if (e != cudaSuccess) {
+    sage::set_error_detail("cudaMallocAsync(scratch)", e);
+    return from_cuda(e);
+  }
+  long long* ksum = static_cast<long long*>(scratch);
+  uint32_t* vmax = reinterpret_cast<uint32_t*>(ksum + n);
+  e = run_prepass(q, k, v, B, H, H_kv, N, d, sm_scale, v_r, q_hat, k_hat, v_hat, delta_q, delta_k,
+                  mean_k, delta_v, ksum, vmax, st);
   cudaError_t ef = cudaFreeAsync(scratch, st);
   return from_cuda(e != cudaSuccess ? e : ef);
 }

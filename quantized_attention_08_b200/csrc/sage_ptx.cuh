@@ -178,6 +178,15 @@ enum : uint32_t { AF_F16 = 0, AF_E4M3 = 0, AF_S8 = 1 };
         "=r"(r[31])                                                                            \
       : "r"(taddr))
 
+#define SAGE_TMEM_LD16(taddr, r)                                                               \
+  asm volatile(                                                                                \
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13," \
+      "%14,%15}, [%16];"                                                                       \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),   \
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),             \
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])                                                  \
+      : "r"(taddr))
+
 #define SAGE_TMEM_ST32(taddr, r)                                                                \
   asm volatile(                                                                                 \
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"   \
@@ -188,6 +197,12 @@ enum : uint32_t { AF_F16 = 0, AF_E4M3 = 0, AF_S8 = 1 };
       "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),       \
       "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),       \
       "r"(r[29]), "r"(r[30]), "r"(r[31]))
+
+#define SAGE_TMEM_ST8(taddr, r)                                                         \
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"( \
+                   taddr),                                                              \
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),   \
+               "r"(r[7]))
 
 #define SAGE_TMEM_ST16(taddr, r)                                                                \
   asm volatile(                                                                                 \
@@ -209,6 +224,16 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+// max of three fp32 values (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Named barrier over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 // Two fp32 -> packed fp16x2 (lo -> bits 0-15), round to nearest even.
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {

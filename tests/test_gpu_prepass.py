@@ -44,6 +44,12 @@ def check_prepass(sage, q, k, v, sm_scale, with_v=True):
         evh9, edv9 = oracle.quant_v_fp8(v, 9.0)
         assert np.array_equal(_bits(dv9.cpu().numpy()), _bits(edv9)), "delta_v (V_r=9)"
         assert np.array_equal(vh9.cpu().numpy(), evh9), "v_hat (V_r=9)"
+        # the combined three-launch pre-pass gives the same bits
+        cq, ck, cdq, cdk, cmk, cvh, cdv = sage.sage_smooth_quant_qkv(tq, tk, tv, sm_scale, 448.0)
+        for got, exp in ((cq, eq), (ck, ekh), (cvh, evh)):
+            assert np.array_equal(got.cpu().numpy(), exp)
+        for got, exp in ((cdq, edq), (cdk, edk), (cmk, emk), (cdv, edv)):
+            assert np.array_equal(_bits(got.cpu().numpy()), _bits(exp))
 
 
 @pytest.mark.parametrize("name", list(workloads.WORKLOADS))
@@ -75,5 +81,6 @@ def test_prepass_degenerate_blocks(sage):
     v = rng.standard_normal((1, 2, 384, 64)).astype(np.float16)
     v[..., 5] = 0                             # zero V column -> delta_v 0
     v[..., 7] = 60000.0                       # large magnitudes
+    v[0, 0, 3, :] = -0.0                      # signed zeros keep their E4M3 sign bit
     k[0, 1, :, 3] = -65504.0                  # extreme fp16 values in the exact mean
     check_prepass(sage, q, k, v, 0.125)

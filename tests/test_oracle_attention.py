@@ -242,3 +242,27 @@ def test_quantized_mirror_accuracy_small(variant):
         assert oracle.rel_l1(o, r) <= 0.02
     else:
         assert oracle.rel_l1(o, r) <= 0.05
+
+
+@pytest.mark.parametrize("variant", ["B", "8+8"])
+def test_ambiguity_slack_bounds_the_flips(variant):
+    """The slack is zero without a band, and bounds the change of the output
+    when every ambiguous operand code takes its other value."""
+    w = workloads.get("llm_8p8_b2_h16_n4096_d128").with_(B=1, H=2, H_kv=1, N=700, causal=True)
+    q, k, v = workloads.generate(w)
+    o0, i0 = oracle.sage_attention(q, k, v, causal=True, variant=variant, ambiguity=0.0,
+                                   simulate_f16acc=False)
+    assert "slack" not in i0
+    eps = 2.0 ** -9   # wide band, so that many codes are ambiguous
+    o1, i1 = oracle.sage_attention(q, k, v, causal=True, variant=variant, ambiguity=eps)
+    assert np.array_equal(o0, o1)
+    slack = i1["slack"]
+    assert np.all(slack >= 0) and slack.max() > 0
+    of, _ = oracle.sage_attention(q, k, v, causal=True, variant=variant, ambiguity=eps,
+                                  flip_ambiguous=True)
+    diff = np.abs(of.astype(np.float64) - o0.astype(np.float64))
+    # both outputs are rounded to fp16: half an ulp each, at most one ulp of the larger
+    big = np.maximum(np.abs(o0), np.abs(of)).astype(np.float16)
+    ulp = np.spacing(big).astype(np.float64)
+    assert np.all(diff <= slack + ulp)
+    assert diff.max() > 0
