@@ -62,6 +62,24 @@ def _peaks():
         return None
 
 
+def max_over_ranks(vals, device=None):
+    """Element-wise max over all ranks of the default process group of a list
+    of floats (identity without a process group or at world size 1).  Every
+    rank must call it, in the same order."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in vals], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tops(ops_per_rank: float, world: int, ms: float) -> float:
+    """Throughput of all ranks together: every rank processes `ops_per_rank`
+    operations, and the job takes the slowest rank's `ms`."""
+    return world * ops_per_rank / (ms * 1e-3) / 1e12
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle sampling during the timed region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -280,13 +298,10 @@ def main():
     total_ms = t_start.elapsed_time(t_end)
     attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
     pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    t = torch.tensor([total_ms, statistics.mean(attn_ms), statistics.mean(pre_ms)],
-                     dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, attn_avg, pre_avg = (float(x) for x in t.tolist())
+    total_ms, attn_avg, pre_avg = max_over_ranks(
+        [total_ms, statistics.mean(attn_ms), statistics.mean(pre_ms)], device=dev)
     ms_per_step = total_ms / args.steps
-    value = world * w.ops / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tops(w.ops, world, ms_per_step)
 
     # end to end through the public one-call API on pinned host buffers
     hq, hk, hv = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
@@ -303,10 +318,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms.append(e0.elapsed_time(e1))
-    te = torch.tensor([statistics.mean(e2e_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * w.ops / (float(te.item()) * 1e-3) / 1e12
+    e2e_avg, = max_over_ranks([statistics.mean(e2e_ms)], device=dev)
+    e2e_value = whole_job_tops(w.ops, world, e2e_avg)
     h2d = (q.nbytes + k.nbytes + v.nbytes)
     d2h = q.nbytes
 
@@ -353,7 +366,7 @@ def main():
                         "algorithmic_bytes": prepass_bytes,
                         "gbs": prepass_bytes / (pre_avg * 1e-3) / 1e9},
             "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": float(te.item())},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_avg},
             "gpu_launches": 4 * args.steps,
             "clocks": {k_: clocks[k_] for k_ in ("sm_mhz", "sm_max_mhz", "reasons")},
             "cpu_baseline": cpu,
