@@ -82,6 +82,37 @@ sage_status_t sage_smooth_quant_qk(const void* q, const void* k, int B, int H, i
                                    float* delta_q, float* delta_k, float* mean_k, void* stream);
 
 /*
+ * sage_smooth_quant_qk without any device allocation.  The paper has no
+ * counterpart: this entry point exists for callers that must not allocate
+ * device memory while they run, for example a serving runtime that plans all
+ * of its device memory up front and treats any allocation after warm-up as an
+ * error, or code that runs where the stream-ordered memory pool of the device
+ * is owned by someone else.  Arguments, layouts and results are those of
+ * sage_smooth_quant_qk, bit for bit.
+ *
+ * Scratch: the int64 partial column sums of K (B*H_kv*ceil(N/256)*d of them)
+ * go to a static array in the library's device memory, 4 MiB per device
+ * (524,288 entries: e.g. B*H_kv = 32 heads of N = 32768 tokens at d = 128).
+ * Larger sizes are rejected with SAGE_ERR_UNSUPPORTED before anything is
+ * launched (sage_last_error_detail() says why); use sage_smooth_quant_qk for
+ * them.  No entry of the array has to start at zero: each call writes every
+ * partial sum it later reads.
+ *
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ * first call before any stream capture begins.
+ *
+ * Concurrency: there is ONE array per device.  Calls issued in order on one
+ * stream are safe; calls that may overlap on the same device (other streams,
+ * other host threads) race on it and can produce wrong results, since the
+ * array keeps whatever the last writer left.  Order such calls with events.
+ */
+sage_status_t sage_smooth_quant_qk_noalloc(const void* q, const void* k, int B, int H,
+                                           int H_kv, int N, int d, float sm_scale,
+                                           int8_t* q_hat, int8_t* k_hat, float* delta_q,
+                                           float* delta_k, float* mean_k, void* stream);
+
+/*
  * FP8 E4M3 quantization of V for the 8+8 variant ([SA2++] delta_V formula and
  * Eq. (2) with a general V_r).
  *   v      : fp16 [B,H_kv,N,d]

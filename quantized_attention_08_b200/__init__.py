@@ -6,7 +6,8 @@ memory and the current stream.  There is no fallback: if the library is not
 built, or the GPU is not a B200, the calls raise.
 
 Functions carry the names of the C entry points:
-  sage_smooth_quant_qk, sage_quant_v_fp8, sage_smooth_quant_qkv,
+  sage_smooth_quant_qk, sage_smooth_quant_qk_noalloc, sage_quant_v_fp8,
+  sage_smooth_quant_qkv,
   sage_attn_fwd_quantized,
   sage_attn_fwd, sage_attn_fwd_ws, sage_attn_workspace_bytes,
   sage_attn_fwd_host, sage_get_device_error, sage_set_wait_timeout_ns,
@@ -36,6 +37,8 @@ _f = _c.c_float
 
 _SIGS = {
     "sage_smooth_quant_qk": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "sage_smooth_quant_qk_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp,
+                                          _vp]),
     "sage_quant_v_fp8": (_i, [_vp, _i, _i, _i, _i, _f, _vp, _vp, _vp]),
     "sage_smooth_quant_qkv": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp, _vp,
                                    _vp, _vp, _vp, _vp]),
@@ -149,6 +152,27 @@ def sage_smooth_quant_qk(q: torch.Tensor, k: torch.Tensor, sm_scale: Optional[fl
                                              _ptr(qh), _ptr(kh), _ptr(dq), _ptr(dk), _ptr(mk),
                                              _stream(stream))
     _check(st, "sage_smooth_quant_qk")
+    return out
+
+
+def sage_smooth_quant_qk_noalloc(q: torch.Tensor, k: torch.Tensor, out,
+                                 sm_scale: Optional[float] = None, stream=None):
+    """sage_smooth_quant_qk with no device allocation inside the call: the
+    caller passes the five output tensors `out` = (q_hat, k_hat, delta_q,
+    delta_k, mean_k) and the library uses its static 4 MiB scratch (sizes
+    with B*H_kv*ceil(N/256)*d > 524288 raise).  Calls that may overlap on
+    one device race on that scratch; see include/sage.h."""
+    _need(q, torch.float16, "q")
+    _need(k, torch.float16, "k")
+    B, H, N, d = q.shape
+    Hk = k.shape[1]
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    qh, kh, dq, dk, mk = out
+    st = load_library().sage_smooth_quant_qk_noalloc(
+        _ptr(q), _ptr(k), B, H, Hk, N, d, float(sm_scale), _ptr(qh), _ptr(kh), _ptr(dq),
+        _ptr(dk), _ptr(mk), _stream(stream))
+    _check(st, "sage_smooth_quant_qk_noalloc")
     return out
 
 

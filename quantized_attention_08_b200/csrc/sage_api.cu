@@ -3,6 +3,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "sage.h"
 #include "sage_internal.h"
@@ -164,6 +165,39 @@ sage_status_t check_fwd_args(const void* q, const void* k, const void* v, void* 
 
 }  // namespace
 
+// ------------------------------------------------ allocation-free pre-pass
+// Scratch of sage_smooth_quant_qk_noalloc: the per-(slab, 256-token chunk,
+// channel) int64 partial sums of K that the column-statistics kernel writes
+// and the finalize kernel reads.  It lives in the module's static device
+// memory (one copy per device, created when the module is loaded), so the
+// call itself never allocates.  Every entry the finalize kernel reads is
+// written earlier in the same call, so nothing here has to start at zero.
+constexpr size_t kNoAllocPartials = size_t(1) << 19;  // 524,288 int64 = 4 MiB
+static __device__ __align__(256) long long g_noalloc_ksum[kNoAllocPartials];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+long long* g_noalloc_ptr[kMaxDevices];  // device address of g_noalloc_ksum, per device
+
+// Set-up, once per device, with that device current.
+sage_status_t noalloc_scratch(int dev, long long** out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_ksum);
+    if (e != cudaSuccess) {
+      sage::set_error_detail("cudaGetSymbolAddress(static pre-pass scratch)", e);
+      return from_cuda(e);
+    }
+    g_noalloc_ptr[dev] = static_cast<long long*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return SAGE_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 sage_status_t sage_smooth_quant_qk(const void* q, const void* k, int B, int H, int H_kv, int N,
@@ -207,6 +241,56 @@ sage_status_t sage_smooth_quant_qk(const void* q, const void* k, int B, int H, i
   }
   cudaError_t ef = cudaFreeAsync(scratch, st);
   return from_cuda(e != cudaSuccess ? e : ef);
+}
+
+sage_status_t sage_smooth_quant_qk_noalloc(const void* q, const void* k, int B, int H, int H_kv,
+                                           int N, int d, float sm_scale, int8_t* q_hat,
+                                           int8_t* k_hat, float* delta_q, float* delta_k,
+                                           float* mean_k, void* stream) {
+  sage_status_t s = check_sizes(B, H, H_kv, N, d);
+  if (s != SAGE_OK) return s;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return SAGE_OK;
+  if (!q || !k || !q_hat || !k_hat || !delta_q || !delta_k || !mean_k) return SAGE_ERR_INVALID_ARG;
+  if (!a16(q) || !a16(k) || !a16(q_hat) || !a16(k_hat) || !a4(delta_q) || !a4(delta_k) ||
+      !a4(mean_k))
+    return SAGE_ERR_MISALIGNED;
+  const int slabs = B * H_kv;
+  const size_t need = static_cast<size_t>(slabs) * sage::stat_chunks(N) * d;
+  if (need > kNoAllocPartials) {
+    sage::set_error_detail(
+        "sage_smooth_quant_qk_noalloc: B*H_kv*ceil(N/256)*d partial sums exceed the static "
+        "scratch of 524288 (4 MiB); use sage_smooth_quant_qk for these sizes",
+        cudaErrorInvalidValue, static_cast<int>(need > 0x7FFFFFFF ? 0x7FFFFFFF : need));
+    return SAGE_ERR_UNSUPPORTED;
+  }
+  if ((s = check_device()) != SAGE_OK) return s;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  long long* ksum = nullptr;
+  if ((s = noalloc_scratch(dev, &ksum)) != SAGE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = sage::launch_colstats(k, nullptr, slabs, N, d, ksum, nullptr, st);
+  if (e == cudaSuccess) e = sage::launch_finalize(ksum, nullptr, slabs, N, d, 0.f, mean_k, nullptr, st);
+  if (e == cudaSuccess) {
+    sage::QuantArgs qa;
+    std::memset(&qa, 0, sizeof(qa));
+    qa.q = q;
+    qa.k = k;
+    qa.q_hat = q_hat;
+    qa.k_hat = k_hat;
+    qa.delta_q = delta_q;
+    qa.delta_k = delta_k;
+    qa.mean_k = mean_k;
+    qa.sm_scale = sm_scale;
+    qa.B = B;
+    qa.H = H;
+    qa.H_kv = H_kv;
+    qa.N = N;
+    qa.d = d;
+    e = sage::launch_quant(qa, st);
+  }
+  return from_cuda(e);
 }
 
 sage_status_t sage_quant_v_fp8(const void* v, int B, int H_kv, int N, int d, float v_r,
