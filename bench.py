@@ -41,18 +41,27 @@ SPEC_8BIT_TOPS = 4500.0          # B200 dense INT8 / FP8 tensor peak, NVIDIA spe
 NOMINAL_8BIT_OVER_BF16 = 2.0     # 4.5 / 2.25 PFLOP/s dense
 
 # DRAM traffic per attention launch from an ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum), keyed by the attention source hash it was taken on;
+# dram__bytes_write.sum), keyed by the attention code hash (_src_hash) it was taken on;
 # reported as null once the kernel source changes.
 NCU_TRAFFIC = {
     # 639.3 MB measured on B=8,H=16,N=8192 (8+8), scaled by elements per tensor
     # (attention DRAM traffic is linear in B*H*N*d once K/V re-reads hit L2)
-    ("950264ac83e970ff", "video_dit_h24_n32768_d128", "8+8"): 479.6e6,
+    ("891d7d4777ebfb5d", "video_dit_h24_n32768_d128", "8+8"): 479.6e6,
+    # 640.1 MB on the same small case for the current source
+    ("8b3547b8b2862944", "video_dit_h24_n32768_d128", "8+8"): 480.1e6,
 }
 
 
 def _src_hash() -> str:
+    """sha256[:16] of the attention kernel source with comments and blank
+    lines removed, so that a comment edit keeps its measured traffic."""
+    import re
     p = os.path.join(ROOT, "quantized_attention_08_b200", "csrc", "attn_sm100.cu")
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+    src = open(p, encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    code = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def _peaks():

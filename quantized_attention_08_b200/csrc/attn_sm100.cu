@@ -15,20 +15,25 @@
 //               max m and sum l in registers, hands the row's rescale factor
 //               alpha = 2^(m_old - m_new) to the correction warps through
 //               shared memory right after the row max (so the rescale of O
-//               overlaps the exponentials), and writes P~ (fp16, or e4m3 of
-//               448 P~) back into the TMEM columns of S.
+//               overlaps the exponentials), and writes P~: fp16 P~ back into
+//               the TMEM columns of S (variant B), or e4m3 of 448 P~ into a
+//               shared-memory tile (8+8).  In the 8+8 kernel S_g(j+1) is
+//               computed while the softmax of S_g(j) runs: the softmax frees
+//               the TMEM columns of S_g as soon as it has loaded them.
 //   warps 8-11  correction: rescale the rows of O_g in TMEM by alpha before
 //               the next P~V accumulates into them, and the epilogue
 //               (O / l, x delta_v[c] / 448 for 8+8, fp16 store).
 //   warp 12     MMA issuer (one thread): S_g = Q_g K_j^T (kind::i8, s32 in
-//               TMEM) and O_g += P_g V_j (kind::f16 / kind::f8f6f4, P_g from TMEM).
+//               TMEM) and O_g += P_g V_j (kind::f16 with P_g from TMEM, or
+//               kind::f8f6f4 with P_g from shared memory).
 //   warp 13     TMA producer (Q once, then K_j, V_j per ring stage).
 //   warps 14-15 idle (complete the last warpgroup for setmaxnreg).
-// Registers: launched at 128 per thread; the softmax warpgroups grow to 192,
-// the correction warpgroup shrinks to 72 and the last warpgroup to 56
-// (8*192 + 4*72 + 4*56 = 16*128 per lane; per SM sub-partition 192+192+72+56).
+// Registers: launched at 128 per thread; setmaxnreg then gives the softmax
+// warpgroups 192 (B) or 184 (8+8), the correction warpgroup 56 / 72 and the
+// last warpgroup 72 / 64, within the 16*128 per lane the launch provides.
 // Tensor memory (512 columns x 128 lanes): S_0 [0,128), S_1 [128,256),
-// O_0 [256,256+d), O_1 [384,384+d); P_g aliases the first columns of S_g.
+// O_0 [256,256+d), O_1 [384,384+d); variant B's P_g aliases the first
+// columns of S_g.
 // Every wait is bounded (see mbar_wait); on expiry the CTA records the
 // error, abandons its work, drains its in-flight copies and MMAs, frees
 // tensor memory and exits.
@@ -43,7 +48,13 @@ namespace sage {
 constexpr int kBM = 128, kBN = 128;
 constexpr int kMmaWarp = 12, kProducerWarp = 13;  // warps 8-11: correction
 constexpr int kAttnThreads = 512;
-constexpr uint32_t kRegSoftmax = 192, kRegCorr = 72, kRegMisc = 56;
+// setmaxnreg shares per role (softmax, correction, other warps); 8 x soft +
+// 4 x corr + 4 x misc must not exceed 16 x 128 (the launch budget per lane).
+template <int VAR> struct Regs;
+template <> struct Regs<0> { static constexpr uint32_t soft = 192, corr = 56, misc = 72; };
+template <> struct Regs<1> { static constexpr uint32_t soft = 184, corr = 72, misc = 64; };
+static_assert(8 * Regs<0>::soft + 4 * Regs<0>::corr + 4 * Regs<0>::misc <= 16 * 128, "register split");
+static_assert(8 * Regs<1>::soft + 4 * Regs<1>::corr + 4 * Regs<1>::misc <= 16 * 128, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2P448 = 8.807354922057604f;  // log2(448): P operand = 448 * P~
 
@@ -56,7 +67,12 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NS * K_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NS * V_BYTES;       // barriers, 512 B
+  // 8+8: P~ operand tiles in shared memory, one per q tile (K-major e4m3,
+  // 128 rows of 128 keys, 128-byte swizzle)
+  static constexpr bool PS = (VAR == 1);
+  static constexpr int P_TILE = kBM * kBN;
+  static constexpr int OFF_P = OFF_V + NS * V_BYTES;
+  static constexpr int OFF_BAR = OFF_P + (PS ? 2 * P_TILE : 0);  // barriers, 512 B
   static constexpr int OFF_ALPHA = OFF_BAR + 512;            // float [2][128]
   static constexpr int OFF_L = OFF_ALPHA + 2 * 128 * 4;      // float [2][128]
   static constexpr int SMEM = OFF_L + 2 * 128 * 4 + 1024;    // + alignment slack
@@ -204,7 +220,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* o_ready = a_full + 2;    // [2] O_g rescaled for j      (128 correction threads)
   uint64_t* pv_done = o_ready + 2;   // [2] PV_g(j) complete        (MMA commit)
   uint64_t* l_full = pv_done + 2;    // [2] final l_g in smem       (128 softmax threads)
-  uint64_t* mma_done = l_full + 2;
+  uint64_t* s_free = l_full + 2;     // [2] S_g(j) loaded by softmax (128 softmax threads; 8+8)
+  uint64_t* mma_done = s_free + 2;
+  // Parity waits are only sound if no waiter can fall two phases behind the
+  // barrier.  8+8 protocol, per tile g and kv step j:
+  //   s_full(j)  S_g(j+1) needs s_free(j), which the softmax arrives after
+  //              waiting s_full(j).
+  //   s_free(j)  the softmax arrives s_free(j+1) after s_full(j+1), which
+  //              needs the MMA thread to have waited s_free(j).
+  //   p_full(j)  the softmax arrives p_full(j+1) after waiting pv_done(j),
+  //              i.e. after the MMA thread consumed p_full(j).
+  //   pv_done(j) PV_g(j+1) needs p_full(j+1) (softmax past its pv_done(j)
+  //              wait) and o_ready(j+1) (correction past its pv_done(j) wait).
+  //   a_full(j)  the softmax arrives a_full(j+1) after pv_done(j), and PV_g(j)
+  //              is issued only after o_ready(j): the correction has already
+  //              consumed a_full(j) (and read alpha(j) from the shared slot).
+  //   o_ready(j) o_ready(j+1) needs pv_done(j), so the MMA thread has passed
+  //              its o_ready(j) wait.
+  // Variant B gets the same bounds from the order S_g(j+1) after PV_g(j)
+  // (P~ lives in the columns of S).
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
@@ -237,6 +271,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&o_ready[g], 128);
       mbar_init(&pv_done[g], 1);
       mbar_init(&l_full[g], 128);
+      mbar_init(&s_free[g], 128);
     }
     mbar_init(mma_done, 1);
     *s_abort = 0;
@@ -253,13 +288,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp < 8) {
     // ---------------------------------------------------------------- softmax
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Regs<VAR>::soft));
     const int g = warp >> 2, wq = warp & 3;
     const int r = wq * 32 + lane;
     const int qb = qb0 + g;
     if (g == 0 || has1) {
       const int nkv_g = g == 0 ? nkv0 : nkv1;
       const uint32_t tS = tmem + (static_cast<uint32_t>(wq * 32) << 16) + g * 128;
+      const uint32_t sP_g = smem_u32(smem + C::OFF_P) + g * C::P_TILE;
       const float dq_l2e = __fmul_rn(p.dq[static_cast<size_t>(bh) * p.nqb + qb], kLog2e);
       const float* dkp = p.dk + static_cast<size_t>(zkv) * p.nkvb;
       float m = -INFINITY, l = 0.f;
@@ -276,6 +312,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         SAGE_TMEM_LD32(tS + 64, (a + 64));
         SAGE_TMEM_LD32(tS + 96, (a + 96));
         tmem_wait_ld();
+        if (C::PS) {  // S_g's columns may now take S_g(j+1)
+          tc_fence_before();
+          mbar_arrive(&s_free[g]);
+        }
         const int valid = p.N - j * kBN;  // keys left in this tile
         const bool masked = (CAUSAL && j == qb) || valid < kBN;
         const int lim = masked ? min(valid, (CAUSAL && j == qb) ? r + 1 : kBN) : kBN;
@@ -284,21 +324,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float m_new = fmaxf(m, __fmul_rn(static_cast<float>(imax), c));
         const float alpha = ex2_approx(m - m_new);  // 0 on the first tile
         if (j > 0) {
-          // the correction warps rescale O_g while this thread computes P~
+          // the correction warps rescale O_g while this thread computes P~.
+          // 8+8: wait for PV_g(j-1) first; it is issued only once O_g was
+          // rescaled for j-1 (so the alpha slot is free), and it frees the P
+          // tile.  Variant B: S_g(j) was issued after PV_g(j-1), so both
+          // already hold.
+          if (C::PS && !__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[g], (j - 1) & 1, s_abort, tlim, 15)))
+            break;
           s_alpha[g * 128 + r] = alpha;
           mbar_arrive(&a_full[g]);
         }
         const float bias = (VAR == 1) ? (kLog2P448 - m_new) : -m_new;
         const float rs = masked ? tile_exp<VAR, true>(a, c, bias, lim) : tile_exp<VAR, false>(a, c, bias, lim);
-        if (VAR == 0) {
-          SAGE_TMEM_ST32(tS + 0, a);
-          SAGE_TMEM_ST32(tS + 32, (a + 32));
+        l = __fmaf_rn(alpha, l, rs);
+        if (C::PS) {
+          // row r, 16-byte chunk c (keys 16c..16c+15) at the 128-byte-swizzled
+          // position of the K-major operand layout
+          const uint32_t rowp = sP_g + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_shared_v4(rowp + ((c ^ (r & 7)) << 4), a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
+          fence_proxy_async_smem();
         } else {
           SAGE_TMEM_ST32(tS + 0, a);
+          SAGE_TMEM_ST32(tS + 32, (a + 32));
+          tmem_wait_st();
+          tc_fence_before();
         }
-        l = __fmaf_rn(alpha, l, rs);
-        tmem_wait_st();
-        tc_fence_before();
         mbar_arrive(&p_full[g]);
         m = m_new;
       }
@@ -307,7 +359,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp < 12) {
     // ---------------------------------------------------------------- correction + epilogue
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegCorr));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(Regs<VAR>::corr));
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -316,13 +368,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int j = 1; ok && j < nkv; ++j) {
       for (int g = 0; g < 2; ++g) {
         if (g == 0 ? (j >= nkv0) : (!has1 || j >= nkv1)) continue;
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&a_full[g], (j - 1) & 1, s_abort, tlim, 10))) {
+        // O_g must hold the complete PV_g(j-1).  Variant B: implied by the
+        // softmax having seen S_g(j), issued after PV_g(j-1).  8+8: wait.
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&a_full[g], (j - 1) & 1, s_abort, tlim, 10) &&
+                                         (!C::PS || mbar_wait(&pv_done[g], (j - 1) & 1, s_abort, tlim, 14)))) {
           ok = false;
           break;
         }
         const float alpha = s_alpha[g * 128 + r];
-        // O_g holds PV_g(j-1), complete: the softmax saw S_g(j), whose commit
-        // covered every earlier MMA.
+        // O_g holds PV_g(j-1), complete
         if (__any_sync(0xFFFFFFFFu, alpha != 1.f)) {
           tc_fence_after();
           const uint32_t tO = tmem + lane_off + 256 + g * 128;
@@ -378,23 +432,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
   } else {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegMisc));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(Regs<VAR>::misc));
     if (warp == kMmaWarp && lane == 0) {
-      // Issue order per kv step i (two q tiles ping-pong on the tensor core):
+      // Variant B, issue order per kv step i (two q tiles ping-pong on the
+      // tensor core):
       //   S_0(i), PV_1(i-1), S_1(i), PV_0(i)
       // so softmax 0 of step i overlaps PV_1(i-1) + S_1(i) and softmax 1
       // overlaps PV_0(i) + S_0(i+1).  S_g(i+1) overwrites the TMEM columns
       // that PV_g(i) reads P_g from; tcgen05.mma ops issued by one thread
-      // execute in order, so the read precedes the overwrite.  The commit
-      // after S_g(i+1) therefore also certifies that PV_g(i) completed, which
-      // is what lets the correction warps rescale O_g once S_g(i+1) is seen.
+      // execute in order, so the read precedes the overwrite.
+      // The correction warps wait for pv_done_g before touching O_g.
       const uint64_t dQ0 = sdesc(smem_u32(sQ), 16, C::QK_SBO, C::QK_SW);
       const uint64_t dK0 = sdesc(smem_u32(sK), 16, C::QK_SBO, C::QK_SW);
       const uint64_t dV0 = sdesc(smem_u32(sV), C::V_LBO, C::V_SBO, C::V_SW);
+      const uint64_t dP0 = sdesc(smem_u32(smem + C::OFF_P), 16, 1024, SW_128B);
       int k_seen = -1, v_seen = -1;
       auto active = [&](int g, int j) { return g == 0 ? (j < nkv0) : (has1 && j < nkv1); };
       auto issue_s = [&](int g, int j) -> bool {
         if (!active(g, j)) return true;
+        // 8+8: S_g(j) reuses the columns of S_g(j-1) once the softmax has loaded them
+        if (C::PS && j > 0 && !mbar_wait(&s_free[g], (j - 1) & 1, s_abort, tlim, 5)) return false;
         if (k_seen < j) {
           if (!mbar_wait(&k_full[j % NS], (j / NS) & 1, s_abort, tlim, 4)) return false;
           k_seen = j;
@@ -422,10 +479,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int kk = 0; kk < kBN / C::PV_K; ++kk) {
           const uint64_t bd = vd + (kk * C::PV_K * C::V_ROW >> 4);
           const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          if (VAR == 0)
-            mma_f16_ts(tmem + 256 + g * 128, tmem + g * 128 + kk * 8, bd, C::IDESC_PV, acc);
+          if (C::PS)  // P_g: K-major e4m3 in shared memory, 32 keys = 32 bytes per step
+            mma_f8_ss(tmem + 256 + g * 128, dP0 + (g * C::P_TILE >> 4) + kk * 2, bd, C::IDESC_PV, acc);
           else
-            mma_f8_ts(tmem + 256 + g * 128, tmem + g * 128 + kk * 8, bd, C::IDESC_PV, acc);
+            mma_f16_ts(tmem + 256 + g * 128, tmem + g * 128 + kk * 8, bd, C::IDESC_PV, acc);
         }
         tc_commit(&pv_done[g]);
         return true;
@@ -433,17 +490,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool ok = mbar_wait(bar_q, 0, s_abort, tlim, 3);
       ok = ok && issue_s(0, 0) && issue_s(1, 0);
       if (ok) tc_commit(&k_empty[0]);
-      ok = ok && issue_pv(0, 0);
-      for (int i = 1; ok && i < nkv; ++i) {
-        ok = issue_s(0, i) && issue_pv(1, i - 1);
-        if (!ok) break;
-        tc_commit(&v_empty[(i - 1) % NS]);
-        ok = issue_s(1, i);
-        if (!ok) break;
-        tc_commit(&k_empty[i % NS]);
-        ok = issue_pv(0, i);
+      if (C::PS) {
+        // S_g(i+1) is issued as soon as the softmax has loaded S_g(i), so it
+        // is ready when the softmax of step i ends:
+        //   S_0(i+1), S_1(i+1), PV_0(i), PV_1(i)
+        for (int i = 0; ok && i < nkv; ++i) {
+          if (i + 1 < nkv) {
+            ok = issue_s(0, i + 1) && issue_s(1, i + 1);
+            if (!ok) break;
+            tc_commit(&k_empty[(i + 1) % NS]);
+          }
+          ok = issue_pv(0, i) && issue_pv(1, i);
+          if (!ok) break;
+          tc_commit(&v_empty[i % NS]);
+        }
+      } else {
+        ok = ok && issue_pv(0, 0);
+        for (int i = 1; ok && i < nkv; ++i) {
+          ok = issue_s(0, i) && issue_pv(1, i - 1);
+          if (!ok) break;
+          tc_commit(&v_empty[(i - 1) % NS]);
+          ok = issue_s(1, i);
+          if (!ok) break;
+          tc_commit(&k_empty[i % NS]);
+          ok = issue_pv(0, i);
+        }
+        if (ok && issue_pv(1, nkv - 1)) tc_commit(&v_empty[(nkv - 1) % NS]);
       }
-      if (ok && issue_pv(1, nkv - 1)) tc_commit(&v_empty[(nkv - 1) % NS]);
       tc_commit(mma_done);
       drain_wait(mma_done, 0, tlim);
     } else if (warp == kProducerWarp && lane == 0) {
