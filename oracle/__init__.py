@@ -8,6 +8,6 @@ share only the seeded input generator (``workloads``), which holds none of
 the method's arithmetic.
 """
 from .codecs import e4m3_decode, e4m3_encode, e4m3_round, fp16_rne, E4M3_MAX, FP16_MAX
-from .sage import (BLOCK, mean_k, quant_blocks, quant_q, smooth_quant_k, quant_v_fp8,
+from .sage import (BLOCK, rope, mean_k, quant_blocks, quant_q, smooth_quant_k, quant_v_fp8,
                    attention_reference, attention_online, sage_attention,
                    f16acc_product_limit, f16acc_bound_ok, cossim, rel_l1, rmse)

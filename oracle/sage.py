@@ -131,6 +131,33 @@ def quant_v_fp8(v: np.ndarray, v_r: float = 448.0):
 
 
 # --------------------------------------------------------------------------
+# Rotary position embedding before the quantizers ([SA1] implementation
+# detail 1: Q and K are rotated and quantized in one pass; the SageAttention
+# summary page: a kernel fusing RoPE with quantization).
+# --------------------------------------------------------------------------
+
+def rope(x: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """Rotary embedding of fp16 x [..., N, d] in the rotate-half pairing:
+    channel i < d/2 pairs with i + d/2, and at token t with c = cos[t, i],
+    s = sin[t, i] (fp32 tables [N, d/2]):
+        y[i]       = x[i] * c - x[i + d/2] * s
+        y[i + d/2] = x[i + d/2] * c + x[i] * s
+    Each product is rounded to fp32, then the sum, then the result to fp16
+    (the value a separate rotary pass would write back in fp16); the fused
+    pre-pass reproduces exactly this."""
+    d = x.shape[-1]
+    h = d // 2
+    assert cos.shape == (x.shape[-2], h) and sin.shape == cos.shape
+    xf = x.astype(F32)
+    c = cos.astype(F32)
+    s = sin.astype(F32)
+    x1, x2 = xf[..., :h], xf[..., h:]
+    y1 = ((x1 * c).astype(F32) - (x2 * s).astype(F32)).astype(F32)
+    y2 = ((x2 * c).astype(F32) + (x1 * s).astype(F32)).astype(F32)
+    return fp16_rne(np.concatenate([y1, y2], axis=-1).astype(np.float64))
+
+
+# --------------------------------------------------------------------------
 # Attention
 # --------------------------------------------------------------------------
 

@@ -140,3 +140,13 @@ def generate(w: Workload):
     if w.v_var != 1.0:
         v *= f32(math.sqrt(w.v_var))
     return q.astype(np.float16), k.astype(np.float16), v.astype(np.float16)
+
+
+def rope_tables(N: int, d: int, base: float = 10000.0):
+    """cos / sin tables [N, d/2] (float32) of the usual rotary frequencies:
+    angle(t, i) = t * base^(-2i/d), evaluated in float64, rounded once."""
+    i = np.arange(d // 2, dtype=np.float64)
+    theta = base ** (-2.0 * i / d)
+    ang = np.arange(N, dtype=np.float64)[:, None] * theta[None, :]
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
