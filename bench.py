@@ -225,6 +225,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rope", action="store_true",
+                    help="fuse a rotary embedding of Q and K into the pre-pass (tables [N, d/2])")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -265,11 +267,18 @@ def main():
             torch.empty(B, Hk, d, dtype=torch.float32, device=dev) if v8 else None)
     o = torch.empty_like(tq)
     stream = torch.cuda.current_stream()
+    if args.rope:
+        cos_np, sin_np = workloads.rope_tables(N, d)
+        tcos, tsin = torch.from_numpy(cos_np).to(dev), torch.from_numpy(sin_np).to(dev)
 
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        sage.sage_smooth_quant_qkv(tq, tk, tv if v8 else None, w.scale, 448.0, out=outs)
+        if args.rope:
+            sage.sage_smooth_quant_qkv_rope(tq, tk, tcos, tsin, tv if v8 else None, w.scale, 448.0,
+                                            out=outs)
+        else:
+            sage.sage_smooth_quant_qkv(tq, tk, tv if v8 else None, w.scale, 448.0, out=outs)
         if evs:
             evs[1].record(stream)
         qh, kh, dq, dk, _, vh, dv = outs
@@ -363,7 +372,7 @@ def main():
             "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N,
                        "d": w.d, "causal": w.causal, "variant": variant,
                        "global_batch": w.B * world, "seq_len": w.N,
-                       "parallelism": f"replicas x{world}",
+                       "parallelism": f"replicas x{world}", "rope": bool(args.rope),
                        "l2": "inputs exceed L2 (Q,K,V %.0f MB > 126 MB); no flush"
                              % ((q.nbytes + k.nbytes + v.nbytes) / 1e6)},
             "pct_of_spec_8bit_peak": 100.0 * value / world / SPEC_8BIT_TOPS,

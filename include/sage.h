@@ -139,6 +139,27 @@ sage_status_t sage_smooth_quant_qkv(const void* q, const void* k, const void* v,
                                     float* delta_k, float* mean_k, float* delta_v, void* stream);
 
 /*
+ * sage_smooth_quant_qkv with a rotary position embedding of Q and K fused in
+ * front of the quantizers ([SA1] implementation detail 1: Q and K are rotated
+ * and quantized in one pass, with no rotated copy written to HBM; the
+ * SageAttention summary page's fused RoPE + quantization kernel).
+ *   cos_t, sin_t: fp32 [N, d/2] device tables, 16-byte aligned, shared by all
+ *                 batches and heads: row t holds cos/sin of token t's angles.
+ * Rotate-half pairing: channel i < d/2 pairs with i + d/2; with c = cos_t[t,i],
+ * s = sin_t[t,i] (fp32 products, then the sum, each rounded to nearest),
+ *   x'[i]       = fp16( x[i] * c - x[i+d/2] * s )
+ *   x'[i+d/2]   = fp16( x[i+d/2] * c + x[i] * s )
+ * and the results are those of sage_smooth_quant_qkv on the rotated fp16 Q
+ * and K, bit for bit (V is not rotated).  Scratch as sage_smooth_quant_qkv.
+ */
+sage_status_t sage_smooth_quant_qkv_rope(const void* q, const void* k, const void* v,
+                                         const float* cos_t, const float* sin_t, int B, int H,
+                                         int H_kv, int N, int d, float sm_scale, float v_r,
+                                         int8_t* q_hat, int8_t* k_hat, uint8_t* v_hat,
+                                         float* delta_q, float* delta_k, float* mean_k,
+                                         float* delta_v, void* stream);
+
+/*
  * Attention on pre-quantized operands ([SA1] Algorithm 1 steps 3-9, Eq. 4-5):
  * per 128-row q block and ascending 128-key kv tiles,
  *   S = int32(q_hat k_hat^T) * delta_q[i] * delta_k[j]   (tcgen05 kind::i8)

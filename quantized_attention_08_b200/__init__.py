@@ -7,7 +7,7 @@ built, or the GPU is not a B200, the calls raise.
 
 Functions carry the names of the C entry points:
   sage_smooth_quant_qk, sage_smooth_quant_qk_noalloc, sage_quant_v_fp8,
-  sage_smooth_quant_qkv,
+  sage_smooth_quant_qkv, sage_smooth_quant_qkv_rope,
   sage_attn_fwd_quantized,
   sage_attn_fwd, sage_attn_fwd_ws, sage_attn_workspace_bytes,
   sage_attn_fwd_host, sage_get_device_error, sage_set_wait_timeout_ns,
@@ -42,6 +42,8 @@ _SIGS = {
     "sage_quant_v_fp8": (_i, [_vp, _i, _i, _i, _i, _f, _vp, _vp, _vp]),
     "sage_smooth_quant_qkv": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp, _vp,
                                    _vp, _vp, _vp, _vp]),
+    "sage_smooth_quant_qkv_rope": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _vp,
+                                        _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "sage_attn_fwd_quantized": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "sage_attn_workspace_bytes": (_c.c_size_t, [_i, _i, _i, _i, _i, _i]),
     "sage_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
@@ -216,6 +218,40 @@ def sage_smooth_quant_qkv(q, k, v=None, sm_scale: Optional[float] = None, v_r: f
         _ptr(q), _ptr(k), _ptr(v), B, H, Hk, N, d, float(sm_scale), float(v_r), _ptr(qh),
         _ptr(kh), _ptr(vh), _ptr(dq), _ptr(dk), _ptr(mk), _ptr(dv), _stream(stream))
     _check(st, "sage_smooth_quant_qkv")
+    return out
+
+
+def sage_smooth_quant_qkv_rope(q, k, cos_t, sin_t, v=None, sm_scale: Optional[float] = None,
+                               v_r: float = 448.0, out=None, stream=None):
+    """sage_smooth_quant_qkv with rotary embedding of Q and K fused in front
+    of the quantizers; cos_t / sin_t are fp32 CUDA tensors [N, d/2].  Same
+    outputs as sage_smooth_quant_qkv."""
+    _need(q, torch.float16, "q")
+    _need(k, torch.float16, "k")
+    _need(cos_t, torch.float32, "cos_t")
+    _need(sin_t, torch.float32, "sin_t")
+    if v is not None:
+        _need(v, torch.float16, "v")
+    B, H, N, d = q.shape
+    Hk = k.shape[1]
+    if tuple(cos_t.shape) != (N, d // 2) or tuple(sin_t.shape) != (N, d // 2):
+        raise ValueError(f"rotary tables must be [N, d/2] = [{N}, {d // 2}]")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        dev = q.device
+        out = (torch.empty_like(q, dtype=torch.int8), torch.empty_like(k, dtype=torch.int8),
+               torch.empty(B, H, _nb(N), dtype=torch.float32, device=dev),
+               torch.empty(B, Hk, _nb(N), dtype=torch.float32, device=dev),
+               torch.empty(B, Hk, d, dtype=torch.float32, device=dev),
+               None if v is None else torch.empty_like(v, dtype=torch.uint8),
+               None if v is None else torch.empty(B, Hk, d, dtype=torch.float32, device=dev))
+    qh, kh, dq, dk, mk, vh, dv = out
+    st = load_library().sage_smooth_quant_qkv_rope(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(cos_t), _ptr(sin_t), B, H, Hk, N, d, float(sm_scale),
+        float(v_r), _ptr(qh), _ptr(kh), _ptr(vh), _ptr(dq), _ptr(dk), _ptr(mk), _ptr(dv),
+        _stream(stream))
+    _check(st, "sage_smooth_quant_qkv_rope")
     return out
 
 

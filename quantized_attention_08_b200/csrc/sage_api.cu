@@ -83,9 +83,10 @@ WsLayout ws_layout(int B, int H, int H_kv, int N, int d, int variant) {
 cudaError_t run_prepass(const void* q, const void* k, const void* v, int B, int H, int H_kv, int N,
                         int d, float sm_scale, float v_r, int8_t* q_hat, int8_t* k_hat,
                         uint8_t* v_hat, float* delta_q, float* delta_k, float* mean_k,
-                        float* delta_v, long long* ksum, uint32_t* vmax, cudaStream_t st) {
+                        float* delta_v, long long* ksum, uint32_t* vmax, cudaStream_t st,
+                        const float* cos_t = nullptr, const float* sin_t = nullptr) {
   const int slabs = B * H_kv;
-  cudaError_t e = sage::launch_colstats(k, v, slabs, N, d, ksum, v ? vmax : nullptr, st);
+  cudaError_t e = sage::launch_colstats(k, v, slabs, N, d, ksum, v ? vmax : nullptr, st, cos_t, sin_t);
   if (e == cudaSuccess)
     e = sage::launch_finalize(ksum, v ? vmax : nullptr, slabs, N, d, v_r, mean_k, delta_v, st);
   if (e == cudaSuccess) {
@@ -106,6 +107,8 @@ cudaError_t run_prepass(const void* q, const void* k, const void* v, int B, int 
     qa.H_kv = H_kv;
     qa.N = N;
     qa.d = d;
+    qa.cos_t = cos_t;
+    qa.sin_t = sin_t;
     e = sage::launch_quant(qa, st);
   }
   return e;
@@ -356,6 +359,41 @@ sage_status_t sage_smooth_quant_qkv(const void* q, const void* k, const void* v,
   uint32_t* vmax = reinterpret_cast<uint32_t*>(ksum + n);
   e = run_prepass(q, k, v, B, H, H_kv, N, d, sm_scale, v_r, q_hat, k_hat, v_hat, delta_q, delta_k,
                   mean_k, delta_v, ksum, vmax, st);
+  cudaError_t ef = cudaFreeAsync(scratch, st);
+  return from_cuda(e != cudaSuccess ? e : ef);
+}
+
+sage_status_t sage_smooth_quant_qkv_rope(const void* q, const void* k, const void* v,
+                                         const float* cos_t, const float* sin_t, int B, int H,
+                                         int H_kv, int N, int d, float sm_scale, float v_r,
+                                         int8_t* q_hat, int8_t* k_hat, uint8_t* v_hat,
+                                         float* delta_q, float* delta_k, float* mean_k,
+                                         float* delta_v, void* stream) {
+  sage_status_t s = check_sizes(B, H, H_kv, N, d);
+  if (s != SAGE_OK) return s;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  const bool hv = v != nullptr;
+  if (hv && (!(v_r > 0.f) || !(v_r <= 448.f))) return SAGE_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return SAGE_OK;
+  if (!q || !k || !cos_t || !sin_t || !q_hat || !k_hat || !delta_q || !delta_k || !mean_k)
+    return SAGE_ERR_INVALID_ARG;
+  if (hv != (v_hat != nullptr) || hv != (delta_v != nullptr)) return SAGE_ERR_INVALID_ARG;
+  if (!a16(q) || !a16(k) || !a16(cos_t) || !a16(sin_t) || !a16(q_hat) || !a16(k_hat) ||
+      !a4(delta_q) || !a4(delta_k) || !a4(mean_k) || (hv && (!a16(v) || !a16(v_hat) || !a4(delta_v))))
+    return SAGE_ERR_MISALIGNED;
+  if ((s = check_device()) != SAGE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n = static_cast<size_t>(B) * H_kv * sage::stat_chunks(N) * d;
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocAsync(&scratch, n * 12, st);
+  if (e != cudaSuccess) {
+    sage::set_error_detail("cudaMallocAsync(scratch)", e);
+    return from_cuda(e);
+  }
+  long long* ksum = static_cast<long long*>(scratch);
+  uint32_t* vmax = reinterpret_cast<uint32_t*>(ksum + n);
+  e = run_prepass(q, k, v, B, H, H_kv, N, d, sm_scale, v_r, q_hat, k_hat, v_hat, delta_q, delta_k,
+                  mean_k, delta_v, ksum, vmax, st, cos_t, sin_t);
   cudaError_t ef = cudaFreeAsync(scratch, st);
   return from_cuda(e != cudaSuccess ? e : ef);
 }

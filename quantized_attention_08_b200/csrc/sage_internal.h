@@ -22,11 +22,14 @@ struct QuantArgs {
   const float* delta_v;
   float sm_scale;
   int B, H, H_kv, N, d;
+  const float* cos_t = nullptr;  // rotary tables [N, d/2] fp32, or nullptr
+  const float* sin_t = nullptr;
 };
 
 size_t stat_chunks(int N);
 cudaError_t launch_colstats(const void* k, const void* v, int slabs, int N, int D, long long* ksum,
-                            uint32_t* vmax, cudaStream_t st);
+                            uint32_t* vmax, cudaStream_t st, const float* cos_t = nullptr,
+                            const float* sin_t = nullptr);
 cudaError_t launch_finalize(const long long* ksum, const uint32_t* vmax, int slabs, int N, int D,
                             float v_r, float* mean_k, float* delta_v, cudaStream_t st);
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st);

@@ -82,6 +82,14 @@ def test_host_argument_checks_need_no_gpu(lib):
     g = lib.sage_quant_v_fp8
     assert g(fake, 1, 2, 128, 64, 500.0, fake, fake, None) == 1
     assert g(fake, 1, 2, 128, 64, 0.0, fake, fake, None) == 1
+    # rotary pre-pass: tables are required and 16-byte aligned
+    r = lib.sage_smooth_quant_qkv_rope
+    args = lambda cs, sn: (fake, fake, None, cs, sn, 1, 2, 2, 128, 64, 0.125, 448.0,
+                           fake, fake, None, fake, fake, fake, None, None)
+    assert r(*args(None, fake)) == 1
+    assert r(*args(fake, None)) == 1
+    assert r(*args(odd, fake)) == 3
+    assert r(*args(fake, fake)[:5], 1, 2, 2, 128, 96, *args(fake, fake)[10:]) == 2
 
 
 def test_workspace_size_is_consistent(lib):
