@@ -1,7 +1,7 @@
 """Throughput of the SageAttention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--variant B|8+8] [--impl sage|reference]
+                    [--variant B|8+8|8+8-r56] [--rope] [--impl sage|reference]
 
 A step is one pass of the whole hot path over one batch of synthetic input:
 the pre-pass (Smooth K, INT8 quantization of Q*sm_scale and K, E4M3
@@ -49,6 +49,8 @@ NCU_TRAFFIC = {
     ("891d7d4777ebfb5d", "video_dit_h24_n32768_d128", "8+8"): 479.6e6,
     # 640.1 MB on the same small case for the current source
     ("8b3547b8b2862944", "video_dit_h24_n32768_d128", "8+8"): 480.1e6,
+    # 637.5 MB on the same small case for the source with the P_r parameter
+    ("27533816e00f9d15", "video_dit_h24_n32768_d128", "8+8"): 478.1e6,
 }
 
 
@@ -69,6 +71,26 @@ def _peaks():
         return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
     except OSError:
         return None
+
+
+def keep_pool_memory(device_index: int) -> bool:
+    """Keep freed blocks in the device's default stream-ordered memory pool
+    (release threshold = max) so that the library's per-call scratch and
+    workspace allocations reuse memory instead of re-mapping it after every
+    synchronisation (the pool's default threshold of 0 returns freed memory
+    to the driver at each event or stream synchronize).  Returns False if
+    cuda-python is not available."""
+    try:
+        from cuda.bindings import driver as drv
+        from cuda.bindings import runtime as rt
+    except ImportError:
+        return False
+    err, pool = rt.cudaDeviceGetDefaultMemPool(device_index)
+    if err != rt.cudaError_t.cudaSuccess:
+        return False
+    err, = rt.cudaMemPoolSetAttribute(pool, rt.cudaMemPoolAttr.cudaMemPoolAttrReleaseThreshold,
+                                      drv.cuuint64_t(2 ** 64 - 1))
+    return err == rt.cudaError_t.cudaSuccess
 
 
 def max_over_ranks(vals, device=None):
@@ -152,8 +174,9 @@ class OracleSampler:
         t0 = time.perf_counter()
         self.qh, self.dq = oracle.quant_q(q, w.scale)
         self.kh, self.dk, _ = oracle.smooth_quant_k(k)
-        if variant == "8+8":
-            vh, self.dv = oracle.quant_v_fp8(v)
+        self.p_r = 56.0 if variant == "8+8-r56" else 448.0
+        if variant != "B":
+            vh, self.dv = oracle.quant_v_fp8(v, 9.0 if variant == "8+8-r56" else 448.0)
             self.vop, self.operand = oracle.e4m3_decode(vh), "e4m3"
         else:
             self.vop, self.dv, self.operand = v, None, "fp16"
@@ -175,7 +198,7 @@ class OracleSampler:
             t0 = time.perf_counter()
             self.oracle.attention_online(self.qh, self.kh, self.dq, self.dk, self.vop,
                                          causal=w.causal, operand=self.operand, dv=self.dv,
-                                         q_blocks=[qb])
+                                         p_r=self.p_r, q_blocks=[qb])
             rows = min(128, w.N - qb * 128)
             t += time.perf_counter() - t0 + self.t_prepass * rows / w.N
             keys = w.N
@@ -252,12 +275,14 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     sage.load_library()
+    pool_kept = keep_pool_memory(local_rank)
 
     q, k, v = workloads.generate(w)
     tq, tk, tv = (torch.from_numpy(x).to(dev) for x in (q, k, v))
     B, H, N, d = q.shape
     Hk = k.shape[1]
-    v8 = variant == "8+8"
+    v8 = variant != "B"
+    v_r = 9.0 if variant == "8+8-r56" else 448.0
     nb = (N + 127) // 128
     outs = (torch.empty_like(tq, dtype=torch.int8), torch.empty_like(tk, dtype=torch.int8),
             torch.empty(B, H, nb, dtype=torch.float32, device=dev),
@@ -275,10 +300,10 @@ def main():
         if evs:
             evs[0].record(stream)
         if args.rope:
-            sage.sage_smooth_quant_qkv_rope(tq, tk, tcos, tsin, tv if v8 else None, w.scale, 448.0,
+            sage.sage_smooth_quant_qkv_rope(tq, tk, tcos, tsin, tv if v8 else None, w.scale, v_r,
                                             out=outs)
         else:
-            sage.sage_smooth_quant_qkv(tq, tk, tv if v8 else None, w.scale, 448.0, out=outs)
+            sage.sage_smooth_quant_qkv(tq, tk, tv if v8 else None, w.scale, v_r, out=outs)
         if evs:
             evs[1].record(stream)
         qh, kh, dq, dk, _, vh, dv = outs
@@ -367,12 +392,14 @@ def main():
             "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "int8 QK^T + e4m3 PV" if v8 else "int8 QK^T + fp16 PV",
+            "dtype": ("int8 QK^T + e4m3 PV (P_r 56, V_r 9)" if variant == "8+8-r56" else
+                      "int8 QK^T + e4m3 PV" if v8 else "int8 QK^T + fp16 PV"),
             "data": "synthetic (seeded numpy, workload recipe; no dataset)",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N,
                        "d": w.d, "causal": w.causal, "variant": variant,
                        "global_batch": w.B * world, "seq_len": w.N,
                        "parallelism": f"replicas x{world}", "rope": bool(args.rope),
+                       "memory_pool": "release threshold max" if pool_kept else "default",
                        "l2": "inputs exceed L2 (Q,K,V %.0f MB > 126 MB); no flush"
                              % ((q.nbytes + k.nbytes + v.nbytes) / 1e6)},
             "pct_of_spec_8bit_peak": 100.0 * value / world / SPEC_8BIT_TOPS,

@@ -58,7 +58,14 @@ typedef enum {
   SAGE_VARIANT_B = 0,
   /* INT8 Q K^T, P~ and V in FP8 E4M3 ("8+8" of [SA2++]): static delta_P = 1/448,
    * per-channel delta_V = colmax|V| / 448, fp32 accumulator. */
-  SAGE_VARIANT_8P8 = 1
+  SAGE_VARIANT_8P8 = 1,
+  /* 8+8 with the narrowed ranges of [SA2++] Eq. (2) and Table 2, P_r = 56 and
+   * V_r = 9: P operand = e4m3(56 P~), delta_V = colmax|V| / 9.  The [SA2++]
+   * pair is chosen so that an FP16 accumulator cannot overflow; tcgen05 runs
+   * E4M3 MMAs with an fp32 accumulator at the same rate, so the accumulator
+   * here stays fp32 in tensor memory.  Same operand layout as SAGE_VARIANT_8P8
+   * (v_hat must be quantized with v_r = 9 for sage_attn_fwd_quantized). */
+  SAGE_VARIANT_8P8_R56 = 2
 } sage_variant_t;
 
 /*
@@ -166,7 +173,7 @@ sage_status_t sage_smooth_quant_qkv_rope(const void* q, const void* k, const voi
  *   online softmax (running max m, row sum l, rescale of O)
  *   O += P~ V  (variant B: fp16 P~ and fp16 V; 8+8: e4m3(448 P~) and v_hat)
  *   O = O / l  (8+8: times delta_v[c] / 448), rounded to fp16.
- *   v_or_vhat: fp16 V for SAGE_VARIANT_B, E4M3 codes for SAGE_VARIANT_8P8
+ *   v_or_vhat: fp16 V for SAGE_VARIANT_B, E4M3 codes for SAGE_VARIANT_8P8 / _R56
  *   delta_v  : fp32 [B,H_kv,d] for 8+8, ignored (may be NULL) for B
  *   o        : fp16 [B,H,N,d] output
  *   causal   : 0 or 1; square, top-left aligned mask (key t visible to query r iff t <= r)

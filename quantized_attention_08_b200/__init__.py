@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(_PKG, "libsage.so")
 
 SAGE_OK = 0
 SAGE_ERR_DEVICE_TIMEOUT = 6
-VARIANTS = {"B": 0, "8+8": 1}
+VARIANTS = {"B": 0, "8+8": 1, "8+8-r56": 2}
 
 _c = ctypes
 _vp = _c.c_void_p

@@ -39,6 +39,8 @@
 // tensor memory and exits.
 #include <cuda_fp16.h>
 #include <math.h>
+
+#include <cmath>
 #include <stdio.h>
 
 #include "sage_internal.h"
@@ -56,7 +58,6 @@ template <> struct Regs<1> { static constexpr uint32_t soft = 184, corr = 72, mi
 static_assert(8 * Regs<0>::soft + 4 * Regs<0>::corr + 4 * Regs<0>::misc <= 16 * 128, "register split");
 static_assert(8 * Regs<1>::soft + 4 * Regs<1>::corr + 4 * Regs<1>::misc <= 16 * 128, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLog2P448 = 8.807354922057604f;  // log2(448): P operand = 448 * P~
 
 template <int D, int VAR>
 struct Cfg {
@@ -99,6 +100,7 @@ struct AttnKParams {
   __half* o;        // [B*H, N, D]
   int H, Hkv, N, nqb, nkvb;
   uint64_t timeout_ns;
+  float log2_pr;    // 8+8: log2 of the P operand range (P operand = P_r * P~)
 };
 
 // Bounded wait that ignores the abort flag: used to drain in-flight work.
@@ -157,7 +159,7 @@ __device__ __forceinline__ int tile_rowmax(uint32_t (&a)[128], int lim) {
   return max(__vimax3_s32(mx[0], mx[1], mx[2]), max(__vimax3_s32(mx[3], mx[4], mx[5]), max(mx[6], mx[7])));
 }
 // P~ of one tile for this thread's row: p = 2^(acc*c + bias) with
-// c = delta_q * delta_k * log2(e), bias = -m_new (+ log2 448 for 8+8).  `a`
+// c = delta_q * delta_k * log2(e), bias = -m_new (+ log2 P_r for 8+8).  `a`
 // holds the s32 scores on entry and the packed P operand on exit (fp16x2, or
 // 4 x e4m3 per word; lower columns in lower bits).  Returns the row sum of
 // the unrounded P values.
@@ -334,7 +336,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           s_alpha[g * 128 + r] = alpha;
           mbar_arrive(&a_full[g]);
         }
-        const float bias = (VAR == 1) ? (kLog2P448 - m_new) : -m_new;
+        const float bias = (VAR == 1) ? (p.log2_pr - m_new) : -m_new;
         const float rs = masked ? tile_exp<VAR, true>(a, c, bias, lim) : tile_exp<VAR, false>(a, c, bias, lim);
         l = __fmaf_rn(alpha, l, rs);
         if (C::PS) {
@@ -641,6 +643,7 @@ static cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   kp.nqb = (a.N + kBM - 1) / kBM;
   kp.nkvb = (a.N + kBN - 1) / kBN;
   kp.timeout_ns = a.timeout_ns;
+  kp.log2_pr = static_cast<float>(std::log2(static_cast<double>(a.p_r)));
   dim3 grid((kp.nqb + 1) / 2, a.B * a.H);
   kern<<<grid, kAttnThreads, C::SMEM, st>>>(tq, tk, tv, kp);
   const cudaError_t e = cudaGetLastError();

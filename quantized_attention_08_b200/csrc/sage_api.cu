@@ -68,13 +68,14 @@ WsLayout ws_layout(int B, int H, int H_kv, int N, int d, int variant) {
   };
   L.q_hat = take(nq * N * d);
   L.k_hat = take(nk * N * d);
-  L.v_hat = take(variant == SAGE_VARIANT_8P8 ? nk * N * d : 0);
+  const bool v8 = variant != SAGE_VARIANT_B;
+  L.v_hat = take(v8 ? nk * N * d : 0);
   L.delta_q = take(nq * nb * 4);
   L.delta_k = take(nk * nb * 4);
   L.mean_k = take(nk * d * 4);
-  L.delta_v = take(variant == SAGE_VARIANT_8P8 ? nk * d * 4 : 0);
+  L.delta_v = take(v8 ? nk * d * 4 : 0);
   L.ksum = take(nk * nchunk * d * 8);
-  L.vmax = take(variant == SAGE_VARIANT_8P8 ? nk * nchunk * d * 4 : 0);
+  L.vmax = take(v8 ? nk * nchunk * d * 4 : 0);
   L.total = off;
   return L;
 }
@@ -118,7 +119,8 @@ cudaError_t run_prepass(const void* q, const void* k, const void* v, int B, int 
 sage_status_t run_forward(const void* q, const void* k, const void* v, void* o, int B, int H,
                           int H_kv, int N, int d, int causal, float sm_scale, int variant,
                           uint8_t* ws, const WsLayout& L, cudaStream_t st) {
-  const bool v8 = variant == SAGE_VARIANT_8P8;
+  const bool v8 = variant != SAGE_VARIANT_B;
+  const bool r56 = variant == SAGE_VARIANT_8P8_R56;
   int8_t* q_hat = reinterpret_cast<int8_t*>(ws + L.q_hat);
   int8_t* k_hat = reinterpret_cast<int8_t*>(ws + L.k_hat);
   uint8_t* v_hat = v8 ? ws + L.v_hat : nullptr;
@@ -129,7 +131,7 @@ sage_status_t run_forward(const void* q, const void* k, const void* v, void* o, 
   long long* ksum = reinterpret_cast<long long*>(ws + L.ksum);
   uint32_t* vmax = v8 ? reinterpret_cast<uint32_t*>(ws + L.vmax) : nullptr;
 
-  cudaError_t e = run_prepass(q, k, v8 ? v : nullptr, B, H, H_kv, N, d, sm_scale, 448.0f, q_hat,
+  cudaError_t e = run_prepass(q, k, v8 ? v : nullptr, B, H, H_kv, N, d, sm_scale, r56 ? 9.0f : 448.0f, q_hat,
                               k_hat, v_hat, delta_q, delta_k, mean_k, delta_v, ksum, vmax, st);
   if (e == cudaSuccess) {
     sage::AttnArgs aa;
@@ -146,7 +148,8 @@ sage_status_t run_forward(const void* q, const void* k, const void* v, void* o, 
     aa.N = N;
     aa.d = d;
     aa.causal = causal;
-    aa.variant = variant;
+    aa.variant = v8 ? 1 : 0;
+    aa.p_r = r56 ? 56.f : 448.f;
     aa.timeout_ns = g_timeout_ns.load();
     e = sage::launch_attention(aa, st);
   }
@@ -157,7 +160,8 @@ sage_status_t check_fwd_args(const void* q, const void* k, const void* v, void* 
                              int H_kv, int N, int d, int causal, float sm_scale, int variant) {
   sage_status_t s = check_sizes(B, H, H_kv, N, d);
   if (s != SAGE_OK) return s;
-  if (variant != SAGE_VARIANT_B && variant != SAGE_VARIANT_8P8) return SAGE_ERR_UNSUPPORTED;
+  if (variant != SAGE_VARIANT_B && variant != SAGE_VARIANT_8P8 && variant != SAGE_VARIANT_8P8_R56)
+    return SAGE_ERR_UNSUPPORTED;
   if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
   if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
   if (B == 0 || N == 0) return SAGE_OK;
@@ -405,11 +409,12 @@ sage_status_t sage_attn_fwd_quantized(const int8_t* q_hat, const int8_t* k_hat,
                                       void* stream) {
   sage_status_t s = check_sizes(B, H, H_kv, N, d);
   if (s != SAGE_OK) return s;
-  if (variant != SAGE_VARIANT_B && variant != SAGE_VARIANT_8P8) return SAGE_ERR_UNSUPPORTED;
+  if (variant != SAGE_VARIANT_B && variant != SAGE_VARIANT_8P8 && variant != SAGE_VARIANT_8P8_R56)
+    return SAGE_ERR_UNSUPPORTED;
   if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
   if (B == 0 || N == 0) return SAGE_OK;
   if (!q_hat || !k_hat || !delta_q || !delta_k || !v_or_vhat || !o) return SAGE_ERR_INVALID_ARG;
-  if (variant == SAGE_VARIANT_8P8 && !delta_v) return SAGE_ERR_INVALID_ARG;
+  if (variant != SAGE_VARIANT_B && !delta_v) return SAGE_ERR_INVALID_ARG;
   if (!a16(q_hat) || !a16(k_hat) || !a16(v_or_vhat) || !a16(o) || !a4(delta_q) || !a4(delta_k) ||
       (delta_v && !a4(delta_v)))
     return SAGE_ERR_MISALIGNED;
@@ -428,7 +433,8 @@ sage_status_t sage_attn_fwd_quantized(const int8_t* q_hat, const int8_t* k_hat,
   aa.N = N;
   aa.d = d;
   aa.causal = causal;
-  aa.variant = variant;
+  aa.variant = variant == SAGE_VARIANT_B ? 0 : 1;
+  aa.p_r = variant == SAGE_VARIANT_8P8_R56 ? 56.f : 448.f;
   aa.timeout_ns = g_timeout_ns.load();
   return from_cuda(sage::launch_attention(aa, static_cast<cudaStream_t>(stream)));
 }
@@ -477,7 +483,8 @@ sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const v
                                  float sm_scale, int variant, void* stream) {
   sage_status_t s = check_sizes(B, H, H_kv, N, d);
   if (s != SAGE_OK) return s;
-  if (variant != SAGE_VARIANT_B && variant != SAGE_VARIANT_8P8) return SAGE_ERR_UNSUPPORTED;
+  if (variant != SAGE_VARIANT_B && variant != SAGE_VARIANT_8P8 && variant != SAGE_VARIANT_8P8_R56)
+    return SAGE_ERR_UNSUPPORTED;
   if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
   if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
   if (B == 0 || N == 0) return SAGE_OK;

@@ -42,8 +42,9 @@ struct AttnArgs {
   const void* v;         // fp16 V (variant B) or e4m3 codes (8+8)
   const float* delta_v;  // 8+8 only
   void* o;               // fp16 [B,H,N,d]
-  int B, H, H_kv, N, d, causal, variant;
+  int B, H, H_kv, N, d, causal, variant;  // variant: 0 = fp16 P~V, 1 = e4m3 P~V
   uint64_t timeout_ns;
+  float p_r = 448.f;  // e4m3 P operand = p_r * P~ (variant 1)
 };
 
 // Returns a cudaError_t; CUDA_ERROR codes of tensor-map encoding are mapped

@@ -49,8 +49,10 @@ def compare_attention(sage, w, variant, q_blocks=None, inputs=None, check_truth=
     o_gpu = gpu_forward(sage, q, k, v, causal=w.causal, sm_scale=w.scale, variant=variant)
     rows = rows_of(w.N, q_blocks)
     o_gpu = o_gpu[:, :, rows]
+    # the narrowed 8+8 ranges (P_r = 56, V_r = 9) are the oracle's 8+8 with those ranges
+    ranges = dict(variant="8+8", v_r=9.0, p_r=56.0) if variant == "8+8-r56" else dict(variant=variant)
     mirror, inter = oracle.sage_attention(q, k, v, causal=w.causal, sm_scale=w.scale,
-                                          variant=variant, q_blocks=q_blocks, ambiguity=EPS_P)
+                                          q_blocks=q_blocks, ambiguity=EPS_P, **ranges)
     slack = inter["slack"]
     assert np.all(np.isfinite(o_gpu))
     err = np.abs(o_gpu.astype(np.float64) - mirror.astype(np.float64))
