@@ -237,6 +237,55 @@ def run_reference(args, w, variant):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """--sweep: the d x N x causal sweep (B*N = 65536 tokens, H = 16), both
+    variants; one JSON line per point with the attention kernel's time (CUDA
+    events, 10 launches after 3 warm-up launches) and the pre-pass time."""
+    import torch
+    import quantized_attention_08_b200 as sage
+    torch.cuda.set_device(0)
+    keep_pool_memory(0)
+    sage.load_library()
+    peaks = _peaks()
+    peak = NOMINAL_8BIT_OVER_BF16 * (peaks["bf16_tflops_sustained"] if peaks else 1400.0)
+    stream = torch.cuda.current_stream()
+    for w in workloads.sweep_workloads():
+        q, k, v = workloads.generate(w)
+        tq, tk, tv = (torch.from_numpy(x).cuda() for x in (q, k, v))
+        for variant in ("B", "8+8"):
+            v8 = variant == "8+8"
+            pre = lambda: sage.sage_smooth_quant_qkv(tq, tk, tv if v8 else None, w.scale, 448.0)
+            qh, kh, dq, dk, _, vh, dv = pre()
+            o = torch.empty_like(tq)
+            attn = lambda: sage.sage_attn_fwd_quantized(qh, kh, dq, dk, vh if v8 else tv,
+                                                        dv if v8 else None, causal=w.causal,
+                                                        variant=variant, o=o)
+            times = {}
+            for name, fn in (("attn", attn), ("prepass", pre)):
+                for _ in range(3):
+                    fn()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                e0.record(stream)
+                for _ in range(10):
+                    fn()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                times[name] = e0.elapsed_time(e1) / 10
+            st, word = sage.sage_get_device_error()
+            assert st == 0, f"device error {word:#x}"
+            tops = w.ops / (times["attn"] * 1e-3) / 1e12
+            print(json.dumps({
+                "sweep": w.name, "variant": variant, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                "causal": w.causal, "attn_ms": times["attn"], "attn_tops": tops,
+                "frac_of_measured": tops / peak, "pct_of_spec": 100.0 * tops / SPEC_8BIT_TOPS,
+                "prepass_ms": times["prepass"],
+                "step_tops": w.ops / ((times["attn"] + times["prepass"]) * 1e-3) / 1e12}),
+                flush=True)
+        del tq, tk, tv, qh, kh, dq, dk, vh, dv, o
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -248,6 +297,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every point of the d x N x causal sweep (one JSON line each)")
     ap.add_argument("--rope", action="store_true",
                     help="fuse a rotary embedding of Q and K into the pre-pass (tables [N, d/2])")
     args = ap.parse_args()
@@ -263,6 +314,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, w, variant)
+        return
+    if args.sweep:
+        if rank == 0:
+            run_sweep(args)
         return
 
     import torch
