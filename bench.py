@@ -51,6 +51,8 @@ NCU_TRAFFIC = {
     ("8b3547b8b2862944", "video_dit_h24_n32768_d128", "8+8"): 480.1e6,
     # 637.5 MB on the same small case for the source with the P_r parameter
     ("27533816e00f9d15", "video_dit_h24_n32768_d128", "8+8"): 478.1e6,
+    # 638.7 MB on the same small case: separate P~V issuer, suspend hint in waits
+    ("9e8c0cd2f7271b7e", "video_dit_h24_n32768_d128", "8+8"): 479.0e6,
 }
 
 

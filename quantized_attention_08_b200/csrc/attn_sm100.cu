@@ -24,10 +24,13 @@
 //               the next P~V accumulates into them, and the epilogue
 //               (O / l, x delta_v[c] / 448 for 8+8, fp16 store).
 //   warp 12     MMA issuer (one thread): S_g = Q_g K_j^T (kind::i8, s32 in
-//               TMEM) and O_g += P_g V_j (kind::f16 with P_g from TMEM, or
-//               kind::f8f6f4 with P_g from shared memory).
+//               TMEM), and for variant B also O_g += P_g V_j (kind::f16,
+//               P_g from TMEM).
 //   warp 13     TMA producer (Q once, then K_j, V_j per ring stage).
-//   warps 14-15 idle (complete the last warpgroup for setmaxnreg).
+//   warp 14     8+8: P~V issuer (one thread): O_g += P_g V_j (kind::f8f6f4,
+//               P_g from shared memory), apart from the S issuer so that
+//               neither waits behind the other.
+//   warp 15     idle (completes the last warpgroup for setmaxnreg).
 // Registers: launched at 128 per thread; setmaxnreg then gives the softmax
 // warpgroups 192 (B) or 184 (8+8), the correction warpgroup 56 / 72 and the
 // last warpgroup 72 / 64, within the 16*128 per lane the launch provides.
@@ -49,6 +52,7 @@ namespace sage {
 
 constexpr int kBM = 128, kBN = 128;
 constexpr int kMmaWarp = 12, kProducerWarp = 13;  // warps 8-11: correction
+constexpr int kPvWarp = 14;  // 8+8: issues the P~V MMAs
 constexpr int kAttnThreads = 512;
 // setmaxnreg shares per role (softmax, correction, other warps); 8 x soft +
 // 4 x corr + 4 x misc must not exceed 16 x 128 (the launch budget per lane).
@@ -224,6 +228,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* l_full = pv_done + 2;    // [2] final l_g in smem       (128 softmax threads)
   uint64_t* s_free = l_full + 2;     // [2] S_g(j) loaded by softmax (128 softmax threads; 8+8)
   uint64_t* mma_done = s_free + 2;
+  uint64_t* pv_mma_done = mma_done + 1;  // end of the PV issuer's MMAs (8+8)
   // Parity waits are only sound if no waiter can fall two phases behind the
   // barrier.  8+8 protocol, per tile g and kv step j:
   //   s_full(j)  S_g(j+1) needs s_free(j), which the softmax arrives after
@@ -241,7 +246,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   //              its o_ready(j) wait.
   // Variant B gets the same bounds from the order S_g(j+1) after PV_g(j)
   // (P~ lives in the columns of S).
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(pv_mma_done + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -276,6 +281,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&s_free[g], 128);
     }
     mbar_init(mma_done, 1);
+    mbar_init(pv_mma_done, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -494,17 +500,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ok) tc_commit(&k_empty[0]);
       if (C::PS) {
         // S_g(i+1) is issued as soon as the softmax has loaded S_g(i), so it
-        // is ready when the softmax of step i ends:
-        //   S_0(i+1), S_1(i+1), PV_0(i), PV_1(i)
-        for (int i = 0; ok && i < nkv; ++i) {
-          if (i + 1 < nkv) {
-            ok = issue_s(0, i + 1) && issue_s(1, i + 1);
-            if (!ok) break;
-            tc_commit(&k_empty[(i + 1) % NS]);
-          }
-          ok = issue_pv(0, i) && issue_pv(1, i);
+        // is ready when the softmax of step i ends; the P~V MMAs come from
+        // their own issuer (warp kPvWarp), so neither waits behind the other.
+        // The two streams touch disjoint TMEM (S vs O) and shared memory.
+        for (int i = 0; ok && i + 1 < nkv; ++i) {
+          ok = issue_s(0, i + 1) && issue_s(1, i + 1);
           if (!ok) break;
-          tc_commit(&v_empty[i % NS]);
+          tc_commit(&k_empty[(i + 1) % NS]);
         }
       } else {
         ok = ok && issue_pv(0, 0);
@@ -521,6 +523,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       tc_commit(mma_done);
       drain_wait(mma_done, 0, tlim);
+    } else if (C::PS && warp == kPvWarp && lane == 0) {
+      // 8+8 P~V issuer: PV_0(i), PV_1(i) per kv step, each once P_g(i) is in
+      // shared memory and O_g has been rescaled for step i.
+      const uint64_t dV0 = sdesc(smem_u32(sV), C::V_LBO, C::V_SBO, C::V_SW);
+      const uint64_t dP0 = sdesc(smem_u32(smem + C::OFF_P), 16, 1024, SW_128B);
+      bool ok = true;
+      for (int i = 0; ok && i < nkv; ++i) {
+        ok = mbar_wait(&v_full[i % NS], (i / NS) & 1, s_abort, tlim, 6);
+        for (int g = 0; ok && g < 2; ++g) {
+          if (!(g == 0 ? (i < nkv0) : (has1 && i < nkv1))) continue;
+          ok = mbar_wait(&p_full[g], i & 1, s_abort, tlim, 7) &&
+               (i == 0 || mbar_wait(&o_ready[g], (i - 1) & 1, s_abort, tlim, 12));
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t vd = dV0 + ((i % NS) * C::V_BYTES >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kBN / C::PV_K; ++kk)
+            mma_f8_ss(tmem + 256 + g * 128, dP0 + (g * C::P_TILE >> 4) + kk * 2,
+                      vd + (kk * C::PV_K * C::V_ROW >> 4), C::IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&pv_done[g]);
+        }
+        if (ok) tc_commit(&v_empty[i % NS]);
+      }
+      tc_commit(pv_mma_done);
+      drain_wait(pv_mma_done, 0, tlim);
     } else if (warp == kProducerWarp && lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
