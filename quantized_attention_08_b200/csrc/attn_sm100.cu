@@ -453,7 +453,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t dQ0 = sdesc(smem_u32(sQ), 16, C::QK_SBO, C::QK_SW);
       const uint64_t dK0 = sdesc(smem_u32(sK), 16, C::QK_SBO, C::QK_SW);
       const uint64_t dV0 = sdesc(smem_u32(sV), C::V_LBO, C::V_SBO, C::V_SW);
-      const uint64_t dP0 = sdesc(smem_u32(smem + C::OFF_P), 16, 1024, SW_128B);
       int k_seen = -1, v_seen = -1;
       auto active = [&](int g, int j) { return g == 0 ? (j < nkv0) : (has1 && j < nkv1); };
       auto issue_s = [&](int g, int j) -> bool {
@@ -473,7 +472,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_commit(&s_full[g]);
         return true;
       };
-      auto issue_pv = [&](int g, int j) -> bool {
+      auto issue_pv = [&](int g, int j) -> bool {  // variant B (P_g from TMEM)
         if (!active(g, j)) return true;
         if (v_seen < j) {
           if (!mbar_wait(&v_full[j % NS], (j / NS) & 1, s_abort, tlim, 6)) return false;
@@ -487,10 +486,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int kk = 0; kk < kBN / C::PV_K; ++kk) {
           const uint64_t bd = vd + (kk * C::PV_K * C::V_ROW >> 4);
           const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          if (C::PS)  // P_g: K-major e4m3 in shared memory, 32 keys = 32 bytes per step
-            mma_f8_ss(tmem + 256 + g * 128, dP0 + (g * C::P_TILE >> 4) + kk * 2, bd, C::IDESC_PV, acc);
-          else
-            mma_f16_ts(tmem + 256 + g * 128, tmem + g * 128 + kk * 8, bd, C::IDESC_PV, acc);
+          mma_f16_ts(tmem + 256 + g * 128, tmem + g * 128 + kk * 8, bd, C::IDESC_PV, acc);
         }
         tc_commit(&pv_done[g]);
         return true;

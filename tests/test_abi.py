@@ -92,6 +92,20 @@ def test_host_argument_checks_need_no_gpu(lib):
     assert r(*args(fake, fake)[:5], 1, 2, 2, 128, 96, *args(fake, fake)[10:]) == 2
 
 
+def test_size_limits_are_rejected_before_any_cuda_call(lib):
+    """The documented limits: B*H <= 65535 (grid.y) and N <= 2^24 (32-bit
+    TMA coordinates); one past each is SAGE_ERR_UNSUPPORTED.  (Only calls
+    that the host checks reject are made: the pointers are fake.)"""
+    f = lib.sage_attn_fwd
+    fake = ctypes.c_void_p(1 << 20)
+    assert f(fake, fake, fake, fake, 1, 65536, 65536, 128, 64, 0, 0.1, 0, None) == 2
+    assert f(fake, fake, fake, fake, 2, 32768, 32768, 128, 64, 0, 0.1, 0, None) == 2
+    assert f(fake, fake, fake, fake, 1, 2, 2, (1 << 24) + 1, 64, 0, 0.1, 0, None) == 2
+    q = lib.sage_smooth_quant_qk
+    assert q(fake, fake, 1, 2, 2, (1 << 24) + 1, 128, 0.1, fake, fake, fake, fake, fake, None) == 2
+    assert lib.sage_attn_workspace_bytes(1, 65536, 65536, 128, 64, 0) == 0
+
+
 def test_workspace_size_is_consistent(lib):
     import quantized_attention_08_b200 as pkg
     a = pkg.sage_attn_workspace_bytes(1, 32, 8, 8192, 128, "B")
