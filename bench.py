@@ -53,6 +53,8 @@ NCU_TRAFFIC = {
     ("27533816e00f9d15", "video_dit_h24_n32768_d128", "8+8"): 478.1e6,
     # 638.7 MB on the same small case: separate P~V issuer, suspend hint in waits
     ("9e8c0cd2f7271b7e", "video_dit_h24_n32768_d128", "8+8"): 479.0e6,
+    # 641.0 MB on the same small case (B-path issuer cleanup)
+    ("ddd20728e76bed3c", "video_dit_h24_n32768_d128", "8+8"): 480.8e6,
 }
 
 

@@ -208,10 +208,14 @@ sage_status_t sage_attn_fwd_ws(const void* q, const void* k, const void* v, void
 
 /*
  * End-to-end call on HOST buffers: copies q, k, v (fp16, host memory; pinned
- * memory gives full PCIe/C2C bandwidth) to the current device, runs
- * sage_attn_fwd, copies o back to host memory and synchronizes `stream`
- * before returning.  Device buffers are stream-ordered allocations freed
- * before return.
+ * memory gives full PCIe/C2C bandwidth and lets copies overlap the kernels)
+ * to the current device, runs the whole pass, copies o back to host memory
+ * and synchronizes `stream` before returning.  The (batch, kv head) units are
+ * processed in up to 4 chunks: copies in run on an internal stream, the
+ * kernels on `stream`, copies out on a second internal stream, so one
+ * chunk's transfers overlap another chunk's kernels.  The results equal
+ * sage_attn_fwd's.  Device buffers are stream-ordered allocations on
+ * `stream`, freed before return.
  */
 sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
                                  void* o_host, int B, int H, int H_kv, int N, int d, int causal,

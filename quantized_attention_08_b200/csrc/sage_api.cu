@@ -491,28 +491,86 @@ sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const v
   if (!q_host || !k_host || !v_host || !o_host) return SAGE_ERR_INVALID_ARG;
   if ((s = check_device()) != SAGE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t qb = static_cast<size_t>(B) * H * N * d * 2;
-  const size_t kb = static_cast<size_t>(B) * H_kv * N * d * 2;
-  const WsLayout L = ws_layout(B, H, H_kv, N, d, variant);
+
+  // The problem splits into independent units, one per (batch, kv head) with
+  // its group of query heads; consecutive units are contiguous in every
+  // tensor.  Chunks of units are pipelined: copies in on one stream, the
+  // pass on `stream`, copies out on a third, so the transfers of one chunk
+  // overlap the kernels of another.
+  const int units = B * H_kv, r = H / H_kv;
+  const int nchunk = units < 4 ? units : 4;
+  const int per = (units + nchunk - 1) / nchunk;
+  const size_t qu = static_cast<size_t>(r) * N * d * 2;  // bytes of one unit of q (and o)
+  const size_t ku = static_cast<size_t>(N) * d * 2;      // bytes of one unit of k (and v)
+  const size_t qb = qu * units, kb = ku * units;
+  const WsLayout L = ws_layout(1, per * r, per, N, d, variant);
   const size_t off_k = align256(qb), off_v = off_k + align256(kb), off_o = off_v + align256(kb);
   const size_t off_ws = off_o + align256(qb);
+
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev[2 * 4 + 2] = {};
+  cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
+  for (int i = 0; e == cudaSuccess && i < 2 * nchunk + 2; ++i)
+    e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+  cudaEvent_t* ev_in = ev;               // [nchunk] inputs of chunk c on the device
+  cudaEvent_t* ev_done = ev + nchunk;    // [nchunk] output of chunk c computed
+  cudaEvent_t ev_alloc = ev[2 * nchunk], ev_out = ev[2 * nchunk + 1];
+
   void* buf = nullptr;
-  cudaError_t e = cudaMallocAsync(&buf, off_ws + L.total, st);
-  if (e != cudaSuccess) return from_cuda(e);
-  uint8_t* base = static_cast<uint8_t*>(buf);
-  e = cudaMemcpyAsync(base, q_host, qb, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(base + off_k, k_host, kb, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(base + off_v, v_host, kb, cudaMemcpyHostToDevice, st);
+  bool allocated = false;
+  if (e == cudaSuccess) e = cudaMallocAsync(&buf, off_ws + L.total, st);
   if (e == cudaSuccess) {
-    s = run_forward(base, base + off_k, base + off_v, base + off_o, B, H, H_kv, N, d, causal,
-                    sm_scale, variant, base + off_ws, L, st);
-    if (s == SAGE_OK)
-      e = cudaMemcpyAsync(o_host, base + off_o, qb, cudaMemcpyDeviceToHost, st);
+    allocated = true;
+    e = cudaEventRecord(ev_alloc, st);
   }
-  cudaError_t ef = cudaFreeAsync(buf, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_alloc, 0);
+  uint8_t* base = static_cast<uint8_t*>(buf);
+  const uint8_t* hq = static_cast<const uint8_t*>(q_host);
+  const uint8_t* hk = static_cast<const uint8_t*>(k_host);
+  const uint8_t* hv = static_cast<const uint8_t*>(v_host);
+  uint8_t* ho = static_cast<uint8_t*>(o_host);
+  for (int c = 0; e == cudaSuccess && c < nchunk; ++c) {
+    const int u0 = c * per, n = (units - u0 < per ? units - u0 : per);
+    if (n <= 0) break;
+    e = cudaMemcpyAsync(base + u0 * qu, hq + u0 * qu, n * qu, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(base + off_k + u0 * ku, hk + u0 * ku, n * ku, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(base + off_v + u0 * ku, hv + u0 * ku, n * ku, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in[c], s_in);
+  }
+  for (int c = 0; e == cudaSuccess && s == SAGE_OK && c < nchunk; ++c) {
+    const int u0 = c * per, n = (units - u0 < per ? units - u0 : per);
+    if (n <= 0) break;
+    e = cudaStreamWaitEvent(st, ev_in[c], 0);
+    if (e != cudaSuccess) break;
+    s = run_forward(base + u0 * qu, base + off_k + u0 * ku, base + off_v + u0 * ku,
+                    base + off_o + u0 * qu, 1, n * r, n, N, d, causal, sm_scale, variant,
+                    base + off_ws, ws_layout(1, n * r, n, N, d, variant), st);
+    if (s == SAGE_OK) e = cudaEventRecord(ev_done[c], st);
+    if (e == cudaSuccess && s == SAGE_OK) e = cudaStreamWaitEvent(s_out, ev_done[c], 0);
+    if (e == cudaSuccess && s == SAGE_OK)
+      e = cudaMemcpyAsync(ho + u0 * qu, base + off_o + u0 * qu, n * qu, cudaMemcpyDeviceToHost, s_out);
+  }
+  // everything on the side streams ends before the buffer is freed on `stream`
+  cudaError_t ec = cudaSuccess;
+  if (s_in) ec = cudaStreamSynchronize(s_in);
+  if (s_out && ec == cudaSuccess) ec = cudaEventRecord(ev_out, s_out);
+  if (s_out && ec == cudaSuccess) ec = cudaStreamWaitEvent(st, ev_out, 0);
+  cudaError_t ef = allocated ? cudaFreeAsync(buf, st) : cudaSuccess;
   cudaError_t es = cudaStreamSynchronize(st);
+  if (s_out) cudaStreamSynchronize(s_out);
+  for (int i = 0; i < 2 * nchunk + 2; ++i)
+    if (ev[i]) cudaEventDestroy(ev[i]);
+  if (s_in) cudaStreamDestroy(s_in);
+  if (s_out) cudaStreamDestroy(s_out);
   if (s != SAGE_OK) return s;
-  if (e != cudaSuccess) return from_cuda(e);
+  if (e != cudaSuccess) {
+    sage::set_error_detail("sage_attn_fwd_host pipeline", e);
+    return from_cuda(e);
+  }
+  if (ec != cudaSuccess) return from_cuda(ec);
   if (ef != cudaSuccess) return from_cuda(ef);
   return from_cuda(es);
 }

@@ -123,6 +123,29 @@ def test_workspace_and_host_entry_points_agree(sage):
         assert torch.equal(o1.cpu(), ho)
 
 
+@pytest.mark.parametrize("shape", [(2, 8, 2, 333, True), (3, 6, 3, 200, False), (1, 24, 24, 130, False)],
+                         ids=["gqa_causal_4units", "9units_3chunks", "24units"])
+def test_host_pipeline_equals_device_path(sage, shape):
+    """sage_attn_fwd_host splits the (batch, kv head) units into chunks whose
+    copies overlap the kernels; the output is sage_attn_fwd's, bit for bit."""
+    B, H, Hk, N, causal = shape
+    w = workloads.get("llm_8p8_b2_h16_n4096_d128").with_(B=B, H=H, H_kv=Hk, N=N, d=64,
+                                                        causal=causal, seed=900 + N)
+    q, k, v = workloads.generate(w)
+    tq, tk, tv = to_dev(q, k, v)
+    hq, hk, hv = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
+    for variant in ("B", "8+8", "8+8-r56"):
+        o1 = sage.sage_attn_fwd(tq, tk, tv, causal=causal, variant=variant)
+        ho = torch.empty(hq.shape, dtype=torch.float16).pin_memory()
+        sage.sage_attn_fwd_host(hq, hk, hv, ho, causal=causal, variant=variant)
+        assert torch.equal(o1.cpu(), ho), variant
+    # pageable host memory works too
+    ho = torch.empty(q.shape, dtype=torch.float16)
+    sage.sage_attn_fwd_host(torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), ho,
+                            causal=causal, variant="8+8")
+    assert torch.equal(sage.sage_attn_fwd(tq, tk, tv, causal=causal, variant="8+8").cpu(), ho)
+
+
 def test_repeated_calls_are_deterministic(sage):
     w = workloads.get("prefill_gqa_causal_h32_kv8_n8192_d128").with_(H=8, H_kv=2, N=2048)
     q, k, v = workloads.generate(w)
