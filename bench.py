@@ -55,6 +55,8 @@ NCU_TRAFFIC = {
     ("9e8c0cd2f7271b7e", "video_dit_h24_n32768_d128", "8+8"): 479.0e6,
     # 641.0 MB on the same small case (B-path issuer cleanup)
     ("ddd20728e76bed3c", "video_dit_h24_n32768_d128", "8+8"): 480.8e6,
+    # 639.6 MB on the same small case (S issuer on warp 15)
+    ("af2d12c4d8fbaca1", "video_dit_h24_n32768_d128", "8+8"): 479.7e6,
 }
 
 

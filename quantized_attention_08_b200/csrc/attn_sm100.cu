@@ -23,14 +23,16 @@
 //   warps 8-11  correction: rescale the rows of O_g in TMEM by alpha before
 //               the next P~V accumulates into them, and the epilogue
 //               (O / l, x delta_v[c] / 448 for 8+8, fp16 store).
-//   warp 12     MMA issuer (one thread): S_g = Q_g K_j^T (kind::i8, s32 in
+//   warp 15     MMA issuer (one thread): S_g = Q_g K_j^T (kind::i8, s32 in
 //               TMEM), and for variant B also O_g += P_g V_j (kind::f16,
-//               P_g from TMEM).
+//               P_g from TMEM); it also allocates and frees the TMEM.
 //   warp 13     TMA producer (Q once, then K_j, V_j per ring stage).
 //   warp 14     8+8: P~V issuer (one thread): O_g += P_g V_j (kind::f8f6f4,
 //               P_g from shared memory), apart from the S issuer so that
 //               neither waits behind the other.
-//   warp 15     idle (completes the last warpgroup for setmaxnreg).
+//   warp 12     idle (completes the last warpgroup for setmaxnreg).  Warp w
+//               runs on sub-partition w % 4: the three helper roles sit on
+//               sub-partitions 1-3 (measured slightly faster than 0-2).
 // Registers: launched at 128 per thread; setmaxnreg then gives the softmax
 // warpgroups 192 (B) or 184 (8+8), the correction warpgroup 56 / 72 and the
 // last warpgroup 72 / 64, within the 16*128 per lane the launch provides.
@@ -51,7 +53,7 @@
 namespace sage {
 
 constexpr int kBM = 128, kBN = 128;
-constexpr int kMmaWarp = 12, kProducerWarp = 13;  // warps 8-11: correction
+constexpr int kMmaWarp = 15, kProducerWarp = 13;  // warps 8-11: correction
 constexpr int kPvWarp = 14;  // 8+8: issues the P~V MMAs
 constexpr int kAttnThreads = 512;
 // setmaxnreg shares per role (softmax, correction, other warps); 8 x soft +
