@@ -236,16 +236,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   //   s_full(j)  S_g(j+1) needs s_free(j), which the softmax arrives after
   //              waiting s_full(j).
   //   s_free(j)  the softmax arrives s_free(j+1) after s_full(j+1), which
-  //              needs the MMA thread to have waited s_free(j).
+  //              needs the S issuer to have waited s_free(j).
   //   p_full(j)  the softmax arrives p_full(j+1) after waiting pv_done(j),
-  //              i.e. after the MMA thread consumed p_full(j).
+  //              i.e. after the P~V issuer consumed p_full(j).
   //   pv_done(j) PV_g(j+1) needs p_full(j+1) (softmax past its pv_done(j)
   //              wait) and o_ready(j+1) (correction past its pv_done(j) wait).
   //   a_full(j)  the softmax arrives a_full(j+1) after pv_done(j), and PV_g(j)
   //              is issued only after o_ready(j): the correction has already
   //              consumed a_full(j) (and read alpha(j) from the shared slot).
-  //   o_ready(j) o_ready(j+1) needs pv_done(j), so the MMA thread has passed
+  //   o_ready(j) o_ready(j+1) needs pv_done(j), so the P~V issuer has passed
   //              its o_ready(j) wait.
+  //   v_full / v_empty, k_full / k_empty: the usual ring, one consumer each
+  //              (the P~V issuer for V, the S issuer for K).
   // Variant B gets the same bounds from the order S_g(j+1) after PV_g(j)
   // (P~ lives in the columns of S).
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(pv_mma_done + 1);
