@@ -34,7 +34,10 @@ design notes of the repository):
     row sum l adds this fp32 P~ before the operand rounding;
   * GQA: query head h reads kv head floor(h * H_kv / H);
   * causal mask is square and top-left aligned (key t visible to query r
-    iff t <= r).
+    iff t <= r);
+  * rotary embedding (when used): rotate-half pairing with caller cos/sin
+    tables [N, d/2], fp32 products and sum, rounded to fp16, then the
+    pre-pass unchanged; the narrowed 8+8 ranges use P_r = 56, V_r = 9.
 """
 from __future__ import annotations
 
