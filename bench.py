@@ -235,7 +235,8 @@ def run_reference(args, w, variant):
         "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy, workload recipe; no dataset)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N, "d": w.d,
-                   "causal": w.causal, "variant": variant},
+                   "causal": w.causal, "variant": variant, "global_batch": w.B, "seq_len": w.N,
+                   "parallelism": "host cores (rank 0 only)"},
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": smp.threads, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
