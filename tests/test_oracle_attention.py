@@ -183,10 +183,10 @@ def test_fp16_accumulator_bound_against_page_values():
     assert oracle.f16acc_product_limit(n) == float(g["product_limit"][0][0])
     p, vv = map(float, g["example_p_v"][0])
     assert oracle.f16acc_bound_ok(p, vv, n)
-    verdict = {}
+    fits = {}
     for p_r, v_r, who in g["table2_pair"]:
-        verdict[(float(p_r), float(v_r))] = oracle.f16acc_bound_ok(float(p_r), float(v_r), n)
-    assert verdict == {(448.0, 448.0): False, (112.0, 4.5): True, (56.0, 9.0): True}
+        fits[(float(p_r), float(v_r))] = oracle.f16acc_bound_ok(float(p_r), float(v_r), n)
+    assert fits == {(448.0, 448.0): False, (112.0, 4.5): True, (56.0, 9.0): True}
     # a 128-wide kv tile summed in one FP16 accumulator: (56, 9) still fits
     assert oracle.f16acc_bound_ok(56.0, 9.0, 128) and not oracle.f16acc_bound_ok(112.0, 9.0, 128)
     # all of 448, 112, 56, 9 and 4.5 are exact E4M3 values
