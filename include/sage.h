@@ -211,7 +211,7 @@ sage_status_t sage_attn_fwd_ws(const void* q, const void* k, const void* v, void
  * memory gives full PCIe/C2C bandwidth and lets copies overlap the kernels)
  * to the current device, runs the whole pass, copies o back to host memory
  * and synchronizes `stream` before returning.  The (batch, kv head) units are
- * processed in up to 4 chunks: copies in run on an internal stream, the
+ * processed in up to 8 chunks: copies in run on an internal stream, the
  * kernels on `stream`, copies out on a second internal stream, so one
  * chunk's transfers overlap another chunk's kernels.  The results equal
  * sage_attn_fwd's.  Device buffers are stream-ordered allocations on

@@ -497,8 +497,9 @@ sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const v
   // tensor.  Chunks of units are pipelined: copies in on one stream, the
   // pass on `stream`, copies out on a third, so the transfers of one chunk
   // overlap the kernels of another.
+  constexpr int kMaxChunks = 8;
   const int units = B * H_kv, r = H / H_kv;
-  const int nchunk = units < 4 ? units : 4;
+  const int nchunk = units < kMaxChunks ? units : kMaxChunks;
   const int per = (units + nchunk - 1) / nchunk;
   const size_t qu = static_cast<size_t>(r) * N * d * 2;  // bytes of one unit of q (and o)
   const size_t ku = static_cast<size_t>(N) * d * 2;      // bytes of one unit of k (and v)
@@ -508,7 +509,7 @@ sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const v
   const size_t off_ws = off_o + align256(qb);
 
   cudaStream_t s_in = nullptr, s_out = nullptr;
-  cudaEvent_t ev[2 * 4 + 2] = {};
+  cudaEvent_t ev[2 * kMaxChunks + 2] = {};
   cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
   for (int i = 0; e == cudaSuccess && i < 2 * nchunk + 2; ++i)
