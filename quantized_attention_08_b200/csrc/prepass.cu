@@ -26,6 +26,7 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "quant_div.h"
 #include "sage_internal.h"
 
 namespace sage {
@@ -223,20 +224,6 @@ __global__ void __launch_bounds__(256) k_finalize(const long long* __restrict__ 
   }
 }
 
-// Correctly rounded x / d given r = RN(1/d) (Markstein's correction step,
-// P. Markstein, "Computation of elementary functions on the IBM RISC
-// System/6000 processor", IBM J. Res. Dev. 34(1), 1990): q = RN(x*r) is
-// within one ulp of x/d, the remainder x - q*d is exact in one fma, and
-// RN(q + rem*r) is the correctly rounded quotient.  Valid away from
-// overflow/underflow, which the quantizer's ranges never reach.  The
-// correction's additions turn a -0 quotient into +0; with d > 0 the quotient
-// carries the sign of x, which copysign restores (E4M3 encodes -0 as 0x80).
-__device__ __forceinline__ float div_rn_by(float x, float d, float r) {
-  const float q = __fmul_rn(x, r);
-  const float rem = __fmaf_rn(-q, d, x);
-  return copysignf(__fmaf_rn(rem, r, q), x);
-}
-
 // Round-half-even of y to an int8 code: adding 1.5*2^23 leaves the rounded
 // integer in the low mantissa bits (the fp32 add rounds to nearest even at
 // unit spacing), whose low byte is the two's-complement code.  No clamp is
@@ -245,14 +232,6 @@ __device__ __forceinline__ float div_rn_by(float x, float d, float r) {
 // -0 and +0 both give code 0.
 __device__ __forceinline__ uint32_t rne_code8(float y) {
   return __float_as_uint(__fadd_rn(y, 12582912.f)) & 0xFFu;
-}
-
-// RN(x / d) given r = RN(1/d) without the sign fix of div_rn_by (for int8
-// codes, where -0 and +0 coincide).
-__device__ __forceinline__ float div_rn_nosign(float x, float d, float r) {
-  const float q = __fmul_rn(x, r);
-  const float rem = __fmaf_rn(-q, d, x);
-  return __fmaf_rn(rem, r, q);
 }
 
 struct QuantJobs {
