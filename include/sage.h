@@ -106,8 +106,11 @@ sage_status_t sage_smooth_quant_qk(const void* q, const void* k, int B, int H, i
  * partial sum it later reads.
  *
  * Set-up: the first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and keeps it; make that
- * first call before any stream capture begins.
+ * (cudaGetSymbolAddress, with that device current) and keeps it for the life
+ * of the process; make that first call before any stream capture begins.
+ * cudaDeviceReset() on that device invalidates the kept address (the
+ * library's device memory is created anew): a process that resets a device
+ * must unload and reload libsage.so before calling this entry point again.
  *
  * Concurrency: there is ONE array per device.  Calls issued in order on one
  * stream are safe; calls that may overlap on the same device (other streams,

@@ -232,7 +232,7 @@ def attention_online(qh, kh, dq, dk, vop, *, causal: bool, operand: str,
     For every such ambiguous element the difference between the two codes,
     times |V operand|, is accumulated (with the same online rescaling as O)
     into a per-output slack; the function then also returns that slack,
-    scaled like O.  flip_ambiguous: use the other code for every ambiguous
+    scaled like O, and each row's final running max m (the row max of S).  flip_ambiguous: use the other code for every ambiguous
     element (checks that the slack bounds the effect).
     Each q block walks its kv tiles in ascending order; with causal only
     tiles j <= i, masking keys t > r on the diagonal tile."""
@@ -243,6 +243,7 @@ def attention_online(qh, kh, dq, dk, vop, *, causal: bool, operand: str,
     rblk = rows // BLOCK
     out = np.zeros((B, H, len(rows), d), dtype=np.float64)
     slack = np.zeros((B, H, len(rows), d), dtype=np.float64)
+    m_final = np.zeros((B, H, len(rows)), dtype=np.float64)
     stats = []
     f16acc_overflow = False
     for b in range(B):
@@ -316,10 +317,12 @@ def attention_online(qh, kh, dq, dk, vop, *, causal: bool, operand: str,
                 scale = 1.0 / l[:, None]
             out[b, h] = O * scale
             slack[b, h] = SL * scale
+            m_final[b, h] = m
     if out_fp16:
         out = fp16_rne(out)
     if return_stats or simulate_f16acc or ambiguity > 0:
-        return out, {"tiles": stats, "f16acc_overflow": f16acc_overflow, "slack": slack}
+        return out, {"tiles": stats, "f16acc_overflow": f16acc_overflow, "slack": slack,
+                     "m": m_final}
     return out
 
 
@@ -352,7 +355,47 @@ def sage_attention(q, k, v, *, causal: bool, sm_scale: Optional[float] = None,
         o, st = o
         inter["f16acc_overflow"] = st["f16acc_overflow"]
         inter["slack"] = st["slack"]
+        inter["m"] = st["m"]
     return o, inter
+
+
+def sage_attention_varlen(q, k, v, cu_seqlens, *, causal: bool, sm_scale: Optional[float] = None,
+                          variant: str = "B", v_r: float = 448.0, p_r: float = 448.0,
+                          q_blocks: Optional[dict] = None, ambiguity: float = 0.0):
+    """A batch of sequences of different lengths packed along the token axis
+    (the SageAttention review's Table 7 runs models whose sequence lengths
+    are not multiples of the block size, e.g. N = 17776 and N = 1105).
+
+    q [H, T, d], k and v [H_kv, T, d]; sequence s holds tokens
+    cu_seqlens[s] .. cu_seqlens[s+1] - 1 of every head.  Every sequence is its
+    own attention problem: its own mean(K), its own 128-token blocks counted
+    from its first token, its own delta_V -- sage_attention on each slice.
+    q_blocks: optional {s: [q block indices of sequence s]} to restrict the
+    output rows (sequences not in the dict are skipped when it is given).
+    Returns (O fp16 [H, T, d] -- rows not computed are zero --, list of the
+    per-sequence intermediates, None for an empty or skipped sequence)."""
+    cu = [int(x) for x in cu_seqlens]
+    assert cu[0] == 0 and all(b >= a for a, b in zip(cu, cu[1:])) and cu[-1] == q.shape[1]
+    out = np.zeros(q.shape, np.float16)
+    slack = np.zeros(q.shape, np.float64)
+    m = np.zeros(q.shape[:2], np.float64)
+    inters = []
+    for s in range(len(cu) - 1):
+        a, b = cu[s], cu[s + 1]
+        if b == a or (q_blocks is not None and s not in q_blocks):
+            inters.append(None)
+            continue
+        blocks = None if q_blocks is None else q_blocks[s]
+        o_s, inter = sage_attention(q[None, :, a:b], k[None, :, a:b], v[None, :, a:b],
+                                    causal=causal, sm_scale=sm_scale, variant=variant, v_r=v_r,
+                                    p_r=p_r, q_blocks=blocks, ambiguity=ambiguity)
+        rows = _rows_from_blocks(b - a, blocks)
+        out[:, a + rows] = o_s[0]
+        if "slack" in inter:
+            slack[:, a + rows] = inter["slack"][0]
+            m[:, a + rows] = inter["m"][0]
+        inters.append(inter)
+    return out, {"per_sequence": inters, "slack": slack, "m": m}
 
 
 # --------------------------------------------------------------------------
