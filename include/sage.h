@@ -180,7 +180,9 @@ sage_status_t sage_smooth_quant_qkv_rope(const void* q, const void* k, const voi
  *   delta_v  : fp32 [B,H_kv,d] for 8+8, ignored (may be NULL) for B
  *   o        : fp16 [B,H,N,d] output
  *   causal   : 0 or 1; square, top-left aligned mask (key t visible to query r iff t <= r)
- * No scratch memory.
+ * The kernel runs one CTA per SM, each walking a fixed list of work items
+ * (two 128-row q blocks of one head); causal lists hold the longest items
+ * first.  No scratch memory.
  */
 sage_status_t sage_attn_fwd_quantized(const int8_t* q_hat, const int8_t* k_hat,
                                       const float* delta_q, const float* delta_k,
@@ -223,6 +225,58 @@ sage_status_t sage_attn_fwd_ws(const void* q, const void* k, const void* v, void
 sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
                                  void* o_host, int B, int H, int H_kv, int N, int d, int causal,
                                  float sm_scale, int variant, void* stream);
+
+/*
+ * Variable-length batches: B sequences of different lengths packed along the
+ * token axis (the models of [SA1] Table 7 have lengths that are not
+ * multiples of the block size, N = 17776 or N = 1105; batching them without
+ * padding means packing).  Every sequence is its own attention problem, with
+ * its own mean(K), its own 128-token blocks counted from its first token and
+ * its own delta_V: the results for sequence b are those of the fixed-length
+ * entry points on that sequence alone (B = 1, N = its length).
+ *   q, o      : fp16 [H, T, d]      k, v : fp16 [H_kv, T, d]
+ *   cu_seqlens: int32 [B+1] in DEVICE memory, non-decreasing, cu_seqlens[0]
+ *               = 0 and cu_seqlens[B] = T: sequence b holds tokens
+ *               cu_seqlens[b] .. cu_seqlens[b+1]-1 of every head
+ *   max_seqlen: host value >= every cu_seqlens[b+1] - cu_seqlens[b]; sizes
+ *               the per-sequence arrays below (nbm = ceil(max_seqlen / 128))
+ *   T         : total tokens (<= 2^30)
+ * Offsets outside [0, T] are clamped and lengths above max_seqlen cut, so
+ * malformed offsets give wrong results for the affected sequences but never
+ * an access outside the tensors.  Causal masks are per sequence (key t
+ * visible to query r of the same sequence iff t <= r).
+ */
+
+/* Pre-pass of a packed batch (sage_smooth_quant_qkv per sequence).
+ *   q_hat: int8 [H, T, d]; k_hat, v_hat: [H_kv, T, d] (v, v_hat, delta_v: all
+ *          NULL for SAGEAttn-B, or all set)
+ *   delta_q: fp32 [B, H, nbm]; delta_k: fp32 [B, H_kv, nbm] (entries past a
+ *          sequence's last block are not written)
+ *   mean_k, delta_v: fp32 [B, H_kv, d]
+ * Scratch: B*H_kv*ceil(max_seqlen/256)*d*12 bytes, stream-ordered. */
+sage_status_t sage_smooth_quant_qkv_varlen(const void* q, const void* k, const void* v,
+                                           const int32_t* cu_seqlens, int B, int max_seqlen, int T,
+                                           int H, int H_kv, int d, float sm_scale, float v_r,
+                                           int8_t* q_hat, int8_t* k_hat, uint8_t* v_hat,
+                                           float* delta_q, float* delta_k, float* mean_k,
+                                           float* delta_v, void* stream);
+
+/* Attention of a packed batch on pre-quantized operands (layouts as written
+ * by sage_smooth_quant_qkv_varlen; v_or_vhat fp16 [H_kv, T, d] for B, E4M3
+ * codes for 8+8).  No scratch memory. */
+sage_status_t sage_attn_fwd_varlen_quantized(const int8_t* q_hat, const int8_t* k_hat,
+                                             const float* delta_q, const float* delta_k,
+                                             const void* v_or_vhat, const float* delta_v, void* o,
+                                             const int32_t* cu_seqlens, int B, int max_seqlen, int T,
+                                             int H, int H_kv, int d, int causal, int variant,
+                                             void* stream);
+
+/* Whole forward pass of a packed batch; intermediates stream-ordered on
+ * `stream` as for sage_attn_fwd. */
+sage_status_t sage_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o,
+                                   const int32_t* cu_seqlens, int B, int max_seqlen, int T, int H,
+                                   int H_kv, int d, int causal, float sm_scale, int variant,
+                                   void* stream);
 
 /* Layout of v_hat: 0 = [B,H_kv,N,d] (same as v).  Always 0 in this library. */
 int sage_v_hat_layout(void);

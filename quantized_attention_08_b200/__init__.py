@@ -10,7 +10,8 @@ Functions carry the names of the C entry points:
   sage_smooth_quant_qkv, sage_smooth_quant_qkv_rope,
   sage_attn_fwd_quantized,
   sage_attn_fwd, sage_attn_fwd_ws, sage_attn_workspace_bytes,
-  sage_attn_fwd_host, sage_get_device_error, sage_set_wait_timeout_ns,
+  sage_attn_fwd_host, sage_smooth_quant_qkv_varlen, sage_attn_fwd_varlen_quantized,
+  sage_attn_fwd_varlen, sage_get_device_error, sage_set_wait_timeout_ns,
   sage_selftest_wait_timeout, sage_status_string, sage_version,
   sage_v_hat_layout.
 """
@@ -49,6 +50,12 @@ _SIGS = {
     "sage_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
     "sage_attn_fwd_ws": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _c.c_size_t, _vp]),
     "sage_attn_fwd_host": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
+    "sage_smooth_quant_qkv_varlen": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _vp,
+                                          _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "sage_attn_fwd_varlen_quantized": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                            _i, _i, _i, _i, _vp]),
+    "sage_attn_fwd_varlen": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i,
+                                  _vp]),
     "sage_v_hat_layout": (_i, []),
     "sage_get_device_error": (_i, [_vp, _c.POINTER(_c.c_uint32)]),
     "sage_set_wait_timeout_ns": (None, [_c.c_uint64]),
@@ -328,6 +335,76 @@ def sage_attn_fwd_host(q_host, k_host, v_host, o_host, *, causal: bool = False,
                                            _variant(variant), _stream(stream))
     _check(st, "sage_attn_fwd_host")
     return o_host
+
+
+def _varlen_shape(q, k, cu_seqlens, max_seqlen):
+    _need(cu_seqlens, torch.int32, "cu_seqlens")
+    H, T, d = q.shape
+    Hk = k.shape[0]
+    B = cu_seqlens.numel() - 1
+    return B, H, Hk, T, d, int(max_seqlen)
+
+
+def sage_smooth_quant_qkv_varlen(q, k, cu_seqlens, max_seqlen: int, v=None,
+                                 sm_scale: Optional[float] = None, v_r: float = 448.0, stream=None):
+    """Pre-pass of a packed batch (q [H,T,d], k/v [H_kv,T,d], cu_seqlens int32
+    [B+1] on the device).  Returns (q_hat, k_hat, delta_q [B,H,nbm],
+    delta_k [B,H_kv,nbm], mean_k [B,H_kv,d], v_hat, delta_v)."""
+    _need(q, torch.float16, "q")
+    _need(k, torch.float16, "k")
+    B, H, Hk, T, d, ms = _varlen_shape(q, k, cu_seqlens, max_seqlen)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    dev = q.device
+    nbm = _nb(ms)
+    qh, kh = torch.empty_like(q, dtype=torch.int8), torch.empty_like(k, dtype=torch.int8)
+    dq = torch.zeros(B, H, nbm, dtype=torch.float32, device=dev)
+    dk = torch.zeros(B, Hk, nbm, dtype=torch.float32, device=dev)
+    mk = torch.empty(B, Hk, d, dtype=torch.float32, device=dev)
+    vh = None if v is None else torch.empty_like(v, dtype=torch.uint8)
+    dv = None if v is None else torch.empty(B, Hk, d, dtype=torch.float32, device=dev)
+    st = load_library().sage_smooth_quant_qkv_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), B, ms, T, H, Hk, d, float(sm_scale),
+        float(v_r), _ptr(qh), _ptr(kh), _ptr(vh), _ptr(dq), _ptr(dk), _ptr(mk), _ptr(dv),
+        _stream(stream))
+    _check(st, "sage_smooth_quant_qkv_varlen")
+    return qh, kh, dq, dk, mk, vh, dv
+
+
+def sage_attn_fwd_varlen_quantized(q_hat, k_hat, delta_q, delta_k, v_or_vhat, delta_v,
+                                   cu_seqlens, max_seqlen: int, *, causal: bool = False,
+                                   variant="B", o=None, stream=None):
+    """Attention of a packed batch on pre-quantized operands; returns o
+    fp16 [H,T,d]."""
+    _need(q_hat, torch.int8, "q_hat")
+    _need(k_hat, torch.int8, "k_hat")
+    var = _variant(variant)
+    B, H, Hk, T, d, ms = _varlen_shape(q_hat, k_hat, cu_seqlens, max_seqlen)
+    if o is None:
+        o = torch.empty(H, T, d, dtype=torch.float16, device=q_hat.device)
+    st = load_library().sage_attn_fwd_varlen_quantized(
+        _ptr(q_hat), _ptr(k_hat), _ptr(delta_q), _ptr(delta_k), _ptr(v_or_vhat), _ptr(delta_v),
+        _ptr(o), _ptr(cu_seqlens), B, ms, T, H, Hk, d, int(bool(causal)), var, _stream(stream))
+    _check(st, "sage_attn_fwd_varlen_quantized")
+    return o
+
+
+def sage_attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen: int, *, causal: bool = False,
+                         sm_scale: Optional[float] = None, variant="B", o=None, stream=None):
+    """Whole forward pass of a packed batch: q [H,T,d], k/v [H_kv,T,d] fp16,
+    cu_seqlens int32 [B+1] on the device; returns o fp16 [H,T,d]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.float16, n)
+    B, H, Hk, T, d, ms = _varlen_shape(q, k, cu_seqlens, max_seqlen)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    st = load_library().sage_attn_fwd_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cu_seqlens), B, ms, T, H, Hk, d,
+        int(bool(causal)), float(sm_scale), _variant(variant), _stream(stream))
+    _check(st, "sage_attn_fwd_varlen")
+    return o
 
 
 def sage_get_device_error(stream=None):

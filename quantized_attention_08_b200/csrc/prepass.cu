@@ -108,8 +108,8 @@ __device__ __forceinline__ uint4 rope8(uint4 x, int t, int cg, const float* __re
 
 template <int D, bool ROPE>
 __global__ void __launch_bounds__(kThreads) k_colstats(const uint4* __restrict__ k,
-                                                       const uint4* __restrict__ v, int N,
-                                                       int nchunk, long long* __restrict__ ksum,
+                                                       const uint4* __restrict__ v, SeqLayout seq,
+                                                       int Hkv, int nchunk, long long* __restrict__ ksum,
                                                        uint32_t* __restrict__ vmax,
                                                        const float* __restrict__ cosT,
                                                        const float* __restrict__ sinT) {
@@ -117,8 +117,12 @@ __global__ void __launch_bounds__(kThreads) k_colstats(const uint4* __restrict__
   constexpr int RPI = kThreads / TPR;    // rows per iteration
   const int chunk = blockIdx.x, slab = blockIdx.y;
   const int cg = threadIdx.x % TPR, rl = threadIdx.x / TPR;
+  size_t row0;
+  int N;  // rows of this slab (token t of the sequence is row row0 + t)
+  slab_rows(seq, slab, Hkv, &row0, &N);
   const int r0 = chunk * kStatRows, r1 = min(N, r0 + kStatRows);
-  const size_t base = static_cast<size_t>(slab) * N * TPR + cg;
+  if (r0 >= N) return;  // a chunk past the end of a short sequence
+  const size_t base = row0 * TPR + cg;
 
   double acc[8];
   uint32_t vm[8];
@@ -191,17 +195,21 @@ __global__ void __launch_bounds__(kThreads) k_colstats(const uint4* __restrict__
 // (lane = channel), then warp 0 combines them.  Integer sums and maxima are
 // exact, so the result does not depend on this order.
 __global__ void __launch_bounds__(256) k_finalize(const long long* __restrict__ ksum,
-                                                  const uint32_t* __restrict__ vmax, int nchunk,
-                                                  int D, int N, float v_r, float* __restrict__ mean_k,
-                                                  float* __restrict__ delta_v) {
+                                                  const uint32_t* __restrict__ vmax, int nchunk_max,
+                                                  int D, SeqLayout seq, int Hkv, float v_r,
+                                                  float* __restrict__ mean_k, float* __restrict__ delta_v) {
   const int slab = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int c = blockIdx.y * 32 + lane;
+  size_t row0;
+  int N;
+  slab_rows(seq, slab, Hkv, &row0, &N);
+  const int nchunk = (N + kStatRows - 1) / kStatRows;  // chunks written for this slab
   __shared__ long long s_s[8][32];
   __shared__ uint32_t s_m[8][32];
   long long s = 0;
   uint32_t m = 0;
   for (int i = w; i < nchunk; i += 8) {
-    const size_t o = (static_cast<size_t>(slab) * nchunk + i) * D + c;
+    const size_t o = (static_cast<size_t>(slab) * nchunk_max + i) * D + c;
     if (ksum != nullptr) s += ksum[o];
     if (vmax != nullptr) m = max(m, vmax[o]);
   }
@@ -214,9 +222,10 @@ __global__ void __launch_bounds__(256) k_finalize(const long long* __restrict__ 
     s += s_s[i][lane];
     m = max(m, s_m[i][lane]);
   }
-  if (ksum != nullptr) {
+  if (ksum != nullptr) {  // an empty sequence has mean 0
     const double sd = __dmul_rn(__ll2double_rn(s), 0x1p-24);
-    mean_k[static_cast<size_t>(slab) * D + c] = __double2float_rn(__ddiv_rn(sd, static_cast<double>(N)));
+    mean_k[static_cast<size_t>(slab) * D + c] =
+        N > 0 ? __double2float_rn(__ddiv_rn(sd, static_cast<double>(N))) : 0.f;
   }
   if (vmax != nullptr) {
     const float cm = __half2float(__ushort_as_half(static_cast<unsigned short>(m)));
@@ -248,7 +257,9 @@ struct QuantJobs {
   float sm_scale;
   const float* cos_t;   // rotary tables [N, D/2] or nullptr
   const float* sin_t;
-  int N, nb;
+  SeqLayout seq;        // rows of each slab
+  int H, Hkv;           // heads of Q, of K and V (slab numbering)
+  int nb;               // 128-token blocks per slab (the longest sequence's)
   int n_q, n_k, n_v;    // number of (slab, block) jobs of each kind
 };
 
@@ -270,8 +281,12 @@ __global__ void __launch_bounds__(kThreads, ROPE ? 3 : 4) k_quant(const QuantJob
     job -= J.n_q + J.n_k;
   }
   const int slab = job / J.nb, blk = job % J.nb;
-  const int rows = min(128, J.N - blk * 128);
-  const size_t row0 = static_cast<size_t>(slab) * J.N + static_cast<size_t>(blk) * 128;
+  size_t srow;
+  int len;
+  slab_rows(J.seq, slab, kind == 0 ? J.H : J.Hkv, &srow, &len);
+  const int rows = min(128, len - blk * 128);
+  if (rows <= 0) return;  // a block past the end of a short sequence
+  const size_t row0 = srow + static_cast<size_t>(blk) * 128;
   const uint4* src = (kind == 0 ? J.q : kind == 1 ? J.k : J.v) + row0 * TPR;
   uint2* dst = (kind == 0 ? J.q_hat : kind == 1 ? J.k_hat : J.v_hat) + row0 * TPR;
   const int cg = threadIdx.x % TPR;  // this thread's 8 channels: cg*8 .. cg*8+7 (fixed across u)
@@ -375,20 +390,32 @@ __global__ void __launch_bounds__(kThreads, ROPE ? 3 : 4) k_quant(const QuantJob
 // ---------------------------------------------------------------- launchers
 size_t stat_chunks(int N) { return static_cast<size_t>((N + kStatRows - 1) / kStatRows); }
 
+// The fixed layout is the packed one's special case of equal lengths
+// (offsets computed instead of read): N rows per slab.
+static SeqLayout fixed_or(SeqLayout seq, int N) {
+  if (seq.cu == nullptr) {
+    seq.T = N;
+    seq.max_len = N;
+  }
+  return seq;
+}
+
 cudaError_t launch_colstats(const void* k, const void* v, int slabs, int N, int D,
                             long long* ksum, uint32_t* vmax, cudaStream_t st, const float* cos_t,
-                            const float* sin_t) {
-  const int nchunk = static_cast<int>(stat_chunks(N));
+                            const float* sin_t, SeqLayout seq, int Hkv) {
+  seq = fixed_or(seq, N);
+  const int nchunk = static_cast<int>(stat_chunks(seq.max_len));
+  if (nchunk == 0 || slabs == 0) return cudaSuccess;
   dim3 grid(nchunk, slabs);
   const uint4* k4 = static_cast<const uint4*>(k);
   const uint4* v4 = static_cast<const uint4*>(v);
   const bool rope = cos_t != nullptr && k != nullptr;
   if (D == 128) {
-    if (rope) k_colstats<128, true><<<grid, kThreads, 0, st>>>(k4, v4, N, nchunk, ksum, vmax, cos_t, sin_t);
-    else k_colstats<128, false><<<grid, kThreads, 0, st>>>(k4, v4, N, nchunk, ksum, vmax, nullptr, nullptr);
+    if (rope) k_colstats<128, true><<<grid, kThreads, 0, st>>>(k4, v4, seq, Hkv, nchunk, ksum, vmax, cos_t, sin_t);
+    else k_colstats<128, false><<<grid, kThreads, 0, st>>>(k4, v4, seq, Hkv, nchunk, ksum, vmax, nullptr, nullptr);
   } else {
-    if (rope) k_colstats<64, true><<<grid, kThreads, 0, st>>>(k4, v4, N, nchunk, ksum, vmax, cos_t, sin_t);
-    else k_colstats<64, false><<<grid, kThreads, 0, st>>>(k4, v4, N, nchunk, ksum, vmax, nullptr, nullptr);
+    if (rope) k_colstats<64, true><<<grid, kThreads, 0, st>>>(k4, v4, seq, Hkv, nchunk, ksum, vmax, cos_t, sin_t);
+    else k_colstats<64, false><<<grid, kThreads, 0, st>>>(k4, v4, seq, Hkv, nchunk, ksum, vmax, nullptr, nullptr);
   }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) set_error_detail("column statistics kernel launch", e);
@@ -396,9 +423,12 @@ cudaError_t launch_colstats(const void* k, const void* v, int slabs, int N, int 
 }
 
 cudaError_t launch_finalize(const long long* ksum, const uint32_t* vmax, int slabs, int N, int D,
-                            float v_r, float* mean_k, float* delta_v, cudaStream_t st) {
-  const int nchunk = static_cast<int>(stat_chunks(N));
-  k_finalize<<<dim3(slabs, D / 32), 256, 0, st>>>(ksum, vmax, nchunk, D, N, v_r, mean_k, delta_v);
+                            float v_r, float* mean_k, float* delta_v, cudaStream_t st, SeqLayout seq,
+                            int Hkv) {
+  seq = fixed_or(seq, N);
+  const int nchunk = static_cast<int>(stat_chunks(seq.max_len));
+  if (slabs == 0) return cudaSuccess;
+  k_finalize<<<dim3(slabs, D / 32), 256, 0, st>>>(ksum, vmax, nchunk, D, seq, Hkv, v_r, mean_k, delta_v);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) set_error_detail("finalize kernel launch", e);
   return e;
@@ -419,8 +449,10 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st) {
   J.sm_scale = a.sm_scale;
   J.cos_t = a.cos_t;
   J.sin_t = a.sin_t;
-  J.N = a.N;
-  J.nb = (a.N + 127) / 128;
+  J.seq = fixed_or(a.seq, a.N);
+  J.H = a.H;
+  J.Hkv = a.H_kv;
+  J.nb = (J.seq.max_len + 127) / 128;
   J.n_q = a.q ? a.B * a.H * J.nb : 0;
   J.n_k = a.k ? a.B * a.H_kv * J.nb : 0;
   J.n_v = a.v ? a.B * a.H_kv * J.nb : 0;

@@ -55,21 +55,26 @@ struct WsLayout {
   size_t q_hat, k_hat, v_hat, delta_q, delta_k, mean_k, delta_v, ksum, vmax, total;
 };
 
-WsLayout ws_layout(int B, int H, int H_kv, int N, int d, int variant) {
+// T < 0: fixed layout ([B, H, N, d]); T >= 0: packed sequences ([H, T, d],
+// at most N tokens each).
+WsLayout ws_layout(int B, int H, int H_kv, int N, int d, int variant, long long T = -1) {
   WsLayout L;
   const size_t nb = static_cast<size_t>((N + 127) / 128);
   const size_t nq = static_cast<size_t>(B) * H, nk = static_cast<size_t>(B) * H_kv;
   const size_t nchunk = sage::stat_chunks(N);
+  // rows of q (and o) and of k (and v): B*H*N and B*H_kv*N, or H*T and H_kv*T
+  const size_t rq = T < 0 ? nq * N : static_cast<size_t>(H) * T;
+  const size_t rk = T < 0 ? nk * N : static_cast<size_t>(H_kv) * T;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
     off += align256(bytes);
     return o;
   };
-  L.q_hat = take(nq * N * d);
-  L.k_hat = take(nk * N * d);
+  L.q_hat = take(rq * d);
+  L.k_hat = take(rk * d);
   const bool v8 = variant != SAGE_VARIANT_B;
-  L.v_hat = take(v8 ? nk * N * d : 0);
+  L.v_hat = take(v8 ? rk * d : 0);
   L.delta_q = take(nq * nb * 4);
   L.delta_k = take(nk * nb * 4);
   L.mean_k = take(nk * d * 4);
@@ -85,11 +90,12 @@ cudaError_t run_prepass(const void* q, const void* k, const void* v, int B, int 
                         int d, float sm_scale, float v_r, int8_t* q_hat, int8_t* k_hat,
                         uint8_t* v_hat, float* delta_q, float* delta_k, float* mean_k,
                         float* delta_v, long long* ksum, uint32_t* vmax, cudaStream_t st,
-                        const float* cos_t = nullptr, const float* sin_t = nullptr) {
+                        const float* cos_t = nullptr, const float* sin_t = nullptr,
+                        sage::SeqLayout seq = sage::SeqLayout()) {
   const int slabs = B * H_kv;
-  cudaError_t e = sage::launch_colstats(k, v, slabs, N, d, ksum, v ? vmax : nullptr, st, cos_t, sin_t);
+  cudaError_t e = sage::launch_colstats(k, v, slabs, N, d, ksum, v ? vmax : nullptr, st, cos_t, sin_t, seq, H_kv);
   if (e == cudaSuccess)
-    e = sage::launch_finalize(ksum, v ? vmax : nullptr, slabs, N, d, v_r, mean_k, delta_v, st);
+    e = sage::launch_finalize(ksum, v ? vmax : nullptr, slabs, N, d, v_r, mean_k, delta_v, st, seq, H_kv);
   if (e == cudaSuccess) {
     sage::QuantArgs qa;
     qa.q = q;
@@ -110,6 +116,7 @@ cudaError_t run_prepass(const void* q, const void* k, const void* v, int B, int 
     qa.d = d;
     qa.cos_t = cos_t;
     qa.sin_t = sin_t;
+    qa.seq = seq;
     e = sage::launch_quant(qa, st);
   }
   return e;
@@ -118,7 +125,8 @@ cudaError_t run_prepass(const void* q, const void* k, const void* v, int B, int 
 // The whole pass with intermediates carved from `ws` (L.total bytes).
 sage_status_t run_forward(const void* q, const void* k, const void* v, void* o, int B, int H,
                           int H_kv, int N, int d, int causal, float sm_scale, int variant,
-                          uint8_t* ws, const WsLayout& L, cudaStream_t st) {
+                          uint8_t* ws, const WsLayout& L, cudaStream_t st,
+                          sage::SeqLayout seq = sage::SeqLayout()) {
   const bool v8 = variant != SAGE_VARIANT_B;
   const bool r56 = variant == SAGE_VARIANT_8P8_R56;
   int8_t* q_hat = reinterpret_cast<int8_t*>(ws + L.q_hat);
@@ -132,7 +140,8 @@ sage_status_t run_forward(const void* q, const void* k, const void* v, void* o, 
   uint32_t* vmax = v8 ? reinterpret_cast<uint32_t*>(ws + L.vmax) : nullptr;
 
   cudaError_t e = run_prepass(q, k, v8 ? v : nullptr, B, H, H_kv, N, d, sm_scale, r56 ? 9.0f : 448.0f, q_hat,
-                              k_hat, v_hat, delta_q, delta_k, mean_k, delta_v, ksum, vmax, st);
+                              k_hat, v_hat, delta_q, delta_k, mean_k, delta_v, ksum, vmax, st, nullptr,
+                              nullptr, seq);
   if (e == cudaSuccess) {
     sage::AttnArgs aa;
     aa.q_hat = q_hat;
@@ -151,6 +160,8 @@ sage_status_t run_forward(const void* q, const void* k, const void* v, void* o, 
     aa.variant = v8 ? 1 : 0;
     aa.p_r = r56 ? 56.f : 448.f;
     aa.timeout_ns = g_timeout_ns.load();
+    aa.cu = seq.cu;
+    aa.T = seq.T;
     e = sage::launch_attention(aa, st);
   }
   return from_cuda(e);
@@ -574,6 +585,133 @@ sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const v
   if (ec != cudaSuccess) return from_cuda(ec);
   if (ef != cudaSuccess) return from_cuda(ef);
   return from_cuda(es);
+}
+
+// ------------------------------------------------ packed variable-length batches
+namespace {
+
+sage_status_t check_varlen(const int32_t* cu, int B, int max_seqlen, int T, int H, int H_kv, int d) {
+  sage_status_t s = check_sizes(B, H, H_kv, max_seqlen, d);
+  if (s != SAGE_OK) return s;
+  if (T < 0) return SAGE_ERR_INVALID_ARG;
+  if (T > (1 << 30)) return SAGE_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
+  if (B > 0 && T > 0 && max_seqlen > 0 && cu == nullptr) return SAGE_ERR_INVALID_ARG;
+  if (cu != nullptr && !a4(cu)) return SAGE_ERR_MISALIGNED;
+  return SAGE_OK;
+}
+
+sage::SeqLayout packed(const int32_t* cu, int max_seqlen, int T) {
+  sage::SeqLayout L;
+  L.cu = cu;
+  L.T = T;
+  L.max_len = max_seqlen;
+  return L;
+}
+
+}  // namespace
+
+sage_status_t sage_smooth_quant_qkv_varlen(const void* q, const void* k, const void* v,
+                                           const int32_t* cu_seqlens, int B, int max_seqlen, int T,
+                                           int H, int H_kv, int d, float sm_scale, float v_r,
+                                           int8_t* q_hat, int8_t* k_hat, uint8_t* v_hat,
+                                           float* delta_q, float* delta_k, float* mean_k,
+                                           float* delta_v, void* stream) {
+  sage_status_t s = check_varlen(cu_seqlens, B, max_seqlen, T, H, H_kv, d);
+  if (s != SAGE_OK) return s;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  const bool hv = v != nullptr;
+  if (hv && (!(v_r > 0.f) || !(v_r <= 448.f))) return SAGE_ERR_INVALID_ARG;
+  if (B == 0 || T == 0 || max_seqlen == 0) return SAGE_OK;
+  if (!q || !k || !q_hat || !k_hat || !delta_q || !delta_k || !mean_k) return SAGE_ERR_INVALID_ARG;
+  if (hv != (v_hat != nullptr) || hv != (delta_v != nullptr)) return SAGE_ERR_INVALID_ARG;
+  if (!a16(q) || !a16(k) || !a16(q_hat) || !a16(k_hat) || !a4(delta_q) || !a4(delta_k) ||
+      !a4(mean_k) || (hv && (!a16(v) || !a16(v_hat) || !a4(delta_v))))
+    return SAGE_ERR_MISALIGNED;
+  if ((s = check_device()) != SAGE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n = static_cast<size_t>(B) * H_kv * sage::stat_chunks(max_seqlen) * d;
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocAsync(&scratch, n * 12, st);
+  if (e != cudaSuccess) {
+    sage::set_error_detail("cudaMallocAsync(scratch)", e);
+    return from_cuda(e);
+  }
+  long long* ksum = static_cast<long long*>(scratch);
+  uint32_t* vmax = reinterpret_cast<uint32_t*>(ksum + n);
+  e = run_prepass(q, k, v, B, H, H_kv, max_seqlen, d, sm_scale, v_r, q_hat, k_hat, v_hat, delta_q,
+                  delta_k, mean_k, delta_v, ksum, vmax, st, nullptr, nullptr,
+                  packed(cu_seqlens, max_seqlen, T));
+  cudaError_t ef = cudaFreeAsync(scratch, st);
+  return from_cuda(e != cudaSuccess ? e : ef);
+}
+
+sage_status_t sage_attn_fwd_varlen_quantized(const int8_t* q_hat, const int8_t* k_hat,
+                                             const float* delta_q, const float* delta_k,
+                                             const void* v_or_vhat, const float* delta_v, void* o,
+                                             const int32_t* cu_seqlens, int B, int max_seqlen, int T,
+                                             int H, int H_kv, int d, int causal, int variant,
+                                             void* stream) {
+  sage_status_t s = check_varlen(cu_seqlens, B, max_seqlen, T, H, H_kv, d);
+  if (s != SAGE_OK) return s;
+  if (variant != SAGE_VARIANT_B && variant != SAGE_VARIANT_8P8 && variant != SAGE_VARIANT_8P8_R56)
+    return SAGE_ERR_UNSUPPORTED;
+  if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
+  if (B == 0 || T == 0 || max_seqlen == 0) return SAGE_OK;
+  if (!q_hat || !k_hat || !delta_q || !delta_k || !v_or_vhat || !o) return SAGE_ERR_INVALID_ARG;
+  if (variant != SAGE_VARIANT_B && !delta_v) return SAGE_ERR_INVALID_ARG;
+  if (!a16(q_hat) || !a16(k_hat) || !a16(v_or_vhat) || !a16(o) || !a4(delta_q) || !a4(delta_k) ||
+      (delta_v && !a4(delta_v)))
+    return SAGE_ERR_MISALIGNED;
+  if ((s = check_device()) != SAGE_OK) return s;
+  sage::AttnArgs aa;
+  aa.q_hat = q_hat;
+  aa.k_hat = k_hat;
+  aa.delta_q = delta_q;
+  aa.delta_k = delta_k;
+  aa.v = v_or_vhat;
+  aa.delta_v = delta_v;
+  aa.o = o;
+  aa.B = B;
+  aa.H = H;
+  aa.H_kv = H_kv;
+  aa.N = max_seqlen;
+  aa.d = d;
+  aa.causal = causal;
+  aa.variant = variant == SAGE_VARIANT_B ? 0 : 1;
+  aa.p_r = variant == SAGE_VARIANT_8P8_R56 ? 56.f : 448.f;
+  aa.timeout_ns = g_timeout_ns.load();
+  aa.cu = cu_seqlens;
+  aa.T = T;
+  return from_cuda(sage::launch_attention(aa, static_cast<cudaStream_t>(stream)));
+}
+
+sage_status_t sage_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o,
+                                   const int32_t* cu_seqlens, int B, int max_seqlen, int T, int H,
+                                   int H_kv, int d, int causal, float sm_scale, int variant,
+                                   void* stream) {
+  sage_status_t s = check_varlen(cu_seqlens, B, max_seqlen, T, H, H_kv, d);
+  if (s != SAGE_OK) return s;
+  if (variant != SAGE_VARIANT_B && variant != SAGE_VARIANT_8P8 && variant != SAGE_VARIANT_8P8_R56)
+    return SAGE_ERR_UNSUPPORTED;
+  if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  if (B == 0 || T == 0 || max_seqlen == 0) return SAGE_OK;
+  if (!q || !k || !v || !o) return SAGE_ERR_INVALID_ARG;
+  if (!a16(q) || !a16(k) || !a16(v) || !a16(o)) return SAGE_ERR_MISALIGNED;
+  if ((s = check_device()) != SAGE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(B, H, H_kv, max_seqlen, d, variant, T);
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, L.total, st);
+  if (e != cudaSuccess) {
+    sage::set_error_detail("cudaMallocAsync(workspace)", e);
+    return from_cuda(e);
+  }
+  s = run_forward(q, k, v, o, B, H, H_kv, max_seqlen, d, causal, sm_scale, variant,
+                  static_cast<uint8_t*>(ws), L, st, packed(cu_seqlens, max_seqlen, T));
+  cudaError_t ef = cudaFreeAsync(ws, st);
+  if (s != SAGE_OK) return s;
+  return from_cuda(ef);
 }
 
 int sage_v_hat_layout(void) { return 0; }
