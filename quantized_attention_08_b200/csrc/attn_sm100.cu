@@ -26,12 +26,6 @@
 //               2^(m_old - m_new) handed to the correction warps, then P~ as
 //               e4m3(448 P~) into a shared-memory operand tile (8+8) or fp16
 //               P~ over the tensor-memory columns of S (variant B).
-//               Warp w and warp w+4 share sub-partition w % 4 and with it
-//               one exp2 unit: their exponential loops take turns (a token
-//               passed through an mbarrier pair), so that one tile's S load,
-//               row max and P~ store overlap the other tile's exponentials.
-//               Part of every row's exponentials runs on the FMA pipe
-//               (exp2_poly2) to relieve the exp2 unit.
 //   warps 8-11  correction: rescale the rows of O_g in tensor memory by alpha
 //               before the next P~V accumulates into them, and the epilogue
 //               (O / l, x delta_v[c] / 448 for 8+8, fp16 store).
@@ -44,11 +38,8 @@
 //   warp 13     TMA producer (Q per item, then K_j, V_j per ring stage).
 //   warp 12     idle (completes the last warpgroup for setmaxnreg).
 // 8+8 look-ahead: the softmax frees the columns of S_g as soon as it has
-// loaded them (after writing the int32 bit pattern of 1.5*2^23 back, which
-// the next S MMA accumulates onto, so that each score arrives as the fp32
-// value 1.5*2^23 + acc and needs one subtraction to become acc), so
-// S_g(j+1) is computed during the softmax of S_g(j).  Variant B keeps P~ in
-// the columns of S: S_g(j+1) waits for P~V_g(j).
+// loaded them, so S_g(j+1) is computed during the softmax of S_g(j).
+// Variant B keeps P~ in the columns of S: S_g(j+1) follows P~V_g(j).
 // Tensor memory (512 columns x 128 lanes): S_0 [0,128), S_1 [128,256),
 // O_0 [256,256+d), O_1 [384,384+d).
 // Every wait is bounded (see mbar_wait); on expiry the CTA records the
@@ -80,22 +71,10 @@ constexpr float kLog2e = 1.4426950408889634f;
 // sum kMagicBits + a reads as the fp32 value 1.5 * 2^23 + a, exactly.
 constexpr uint32_t kMagicBits = 0x4B400000u;
 constexpr float kMagic = 12582912.f;
-// Pairs of columns whose exponentials run on the FMA pipe: bit k set ->
-// columns 16t + 2k, 16t + 2k + 1 of every 16-column group t.
-template <int VAR> struct PolyMask;
-template <> struct PolyMask<0> { static constexpr uint32_t bits = 0x00; };
-template <> struct PolyMask<1> { static constexpr uint32_t bits = 0x00; };
-// Turn-taking of the two softmax warps of a sub-partition on its exp2 unit:
-// `on` enables it; a warp hands the unit over once it has issued the
-// exponentials of `release` columns (128: at the end of its loop).
-template <int VAR> struct Turns;
-template <> struct Turns<0> { static constexpr bool on = true; static constexpr int release = 128; };
-template <> struct Turns<1> { static constexpr bool on = false; static constexpr int release = 128; };
 
 template <int D, int VAR>
 struct Cfg {
   static constexpr bool PS = (VAR == 1);        // P~ through shared memory (8+8)
-  static constexpr bool PREFILL = false;        // S accumulates onto kMagicBits
   static constexpr int PB = 1;                  // P~ (and alpha) buffers per q tile
   static constexpr int LS = PB + 1;             // slots for the final row sums of an item
   static constexpr int NS = (D == 128) ? 3 : 4; // K/V ring stages
@@ -235,41 +214,6 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x for a pair of fp32 values on the FMA pipe.  Range reduction x = n + r
-// with n = rint(x) (the 1.5 * 2^23 addition) and r = x - n in [-1/2, 1/2],
-// exact in fp32; 2^r by a degree-5 polynomial minimising the relative error
-// on [-1/2, 1/2] (coefficients fitted by a Remez exchange,
-// fit_exp2_poly.py; relative error below 2^-22 evaluated in fp32); 2^n is
-// added into the exponent field.  The caller guarantees x >= -124, or sets
-// CLAMP, which raises x to -125 first, so the exponent field cannot wrap
-// (2^-125 stands for anything smaller: it rounds to a zero operand code).
-constexpr float kExpC0 = 1.00000011920928955e+00f;
-constexpr float kExpC1 = 6.93146944046020508e-01f;
-constexpr float kExpC2 = 2.40221202373504639e-01f;
-constexpr float kExpC3 = 5.55071309208869934e-02f;
-constexpr float kExpC4 = 9.67554096132516861e-03f;
-constexpr float kExpC5 = 1.32764724548906088e-03f;
-template <bool CLAMP>
-__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& y0, float& y1) {
-  if (CLAMP) {
-    const float2 x = up2(x2);
-    x2 = pk2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
-  }
-  const uint64_t t2 = add2(x2, pk2(kMagic, kMagic));    // 1.5 * 2^23 + rint(x)
-  const uint64_t n2 = add2(t2, pk2(-kMagic, -kMagic));  // rint(x)
-  const uint64_t r2 = fma2(n2, pk2(-1.f, -1.f), x2);    // x - rint(x)
-  uint64_t q2 = fma2(r2, pk2(kExpC5, kExpC5), pk2(kExpC4, kExpC4));
-  q2 = fma2(q2, r2, pk2(kExpC3, kExpC3));
-  q2 = fma2(q2, r2, pk2(kExpC2, kExpC2));
-  q2 = fma2(q2, r2, pk2(kExpC1, kExpC1));
-  q2 = fma2(q2, r2, pk2(kExpC0, kExpC0));
-  const float2 q = up2(q2), t = up2(t2);
-  // the low bits of t hold rint(x) (two's complement): shifted into the
-  // exponent field they scale q by 2^rint(x)
-  y0 = __uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23));
-  y1 = __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23));
-}
-
 // Row max of the s32 scores of one tile (columns >= lim masked when MASKED):
 // eight independent 3-input chains, then a tree.
 template <bool MASKED>
@@ -292,32 +236,29 @@ __device__ __forceinline__ int tile_rowmax(uint32_t (&a)[128], int lim) {
   return max(__vimax3_s32(mx[0], mx[1], mx[2]), max(__vimax3_s32(mx[3], mx[4], mx[5]), max(mx[6], mx[7])));
 }
 
-// P~ of columns [C0, C1) of one tile for this thread's row: p = 2^(acc*c +
-// bias) with c = delta_q * delta_k * log2(e), bias = -m_new (+ log2 P_r for
-// 8+8); c2, b2 hold (c, c) and (bias, bias).  `a` holds the s32 scores on
-// entry (kMagicBits + acc when PREFILL) and the packed P operand on exit
-// (fp16x2, or 4 x e4m3 per word; lower columns in lower bits).  The
-// unrounded P values are added to the four packed partial row sums sum2.
-template <int VAR, bool MASKED, bool PREFILL, bool CLAMP, int C0, int C1>
-__device__ __forceinline__ void tile_exp(uint32_t (&a)[128], uint64_t c2, uint64_t b2, int lim,
-                                         uint64_t (&sum2)[4]) {
-  const uint64_t magic2 = pk2(-kMagic, -kMagic);
+// P~ of one tile for this thread's row: p = 2^(acc*c + bias) with
+// c = delta_q * delta_k * log2(e), bias = -m_new (+ log2 P_r for 8+8).  `a`
+// holds the s32 scores on entry and the packed P operand on exit (fp16x2, or
+// 4 x e4m3 per word; lower columns in lower bits).  Returns the row sum of
+// the unrounded P values.
+template <int VAR, bool MASKED>
+__device__ __forceinline__ float tile_exp(uint32_t (&a)[128], float c, float bias, int lim) {
+  const uint64_t c2 = pk2(c, c), b2 = pk2(bias, bias), magic2 = pk2(-kMagic, -kMagic);
+  uint64_t sum2[4];
 #pragma unroll
-  for (int i = C0; i < C1; i += 4) {
+  for (int t = 0; t < 4; ++t) sum2[t] = 0;
+#pragma unroll
+  for (int i = 0; i < 128; i += 4) {
     float p[4];
 #pragma unroll
     for (int e = 0; e < 4; e += 2) {
-      const uint32_t b0 = PREFILL ? a[i + e] : a[i + e] + kMagicBits;
-      const uint32_t b1 = PREFILL ? a[i + e + 1] : a[i + e + 1] + kMagicBits;
-      const uint64_t f2 = add2(pk2(__uint_as_float(b0), __uint_as_float(b1)), magic2);  // acc, exact
-      const uint64_t x2 = fma2(f2, c2, b2);
-      if ((PolyMask<VAR>::bits >> (((i + e) & 15) >> 1)) & 1u) {
-        exp2_poly2<CLAMP>(x2, p[e], p[e + 1]);
-      } else {
-        const float2 x = up2(x2);
-        p[e] = ex2_approx(x.x);
-        p[e + 1] = ex2_approx(x.y);
-      }
+      // kMagicBits + acc reads as the fp32 value 1.5 * 2^23 + acc: one
+      // subtraction gives acc exactly
+      const uint64_t f2 = add2(pk2(__uint_as_float(a[i + e] + kMagicBits), __uint_as_float(a[i + e + 1] + kMagicBits)),
+                               magic2);
+      const float2 x = up2(fma2(f2, c2, b2));
+      p[e] = ex2_approx(x.x);
+      p[e + 1] = ex2_approx(x.y);
       if (MASKED) {
         if (i + e >= lim) p[e] = 0.f;
         if (i + e + 1 >= lim) p[e + 1] = 0.f;
@@ -331,38 +272,8 @@ __device__ __forceinline__ void tile_exp(uint32_t (&a)[128], uint64_t c2, uint64
       a[i / 4] = pack_e4m3x2(p[0], p[1]) | (pack_e4m3x2(p[2], p[3]) << 16);
     }
   }
-}
-
-// The whole tile: columns [0, R), then the hand-over of the exp2 unit
-// (`release`, one lane arrives on `tok` once the warp got there), then
-// [R, 128).  Returns the row sum of the unrounded P values.
-template <int VAR, bool MASKED, bool PREFILL, bool CLAMP, int R>
-__device__ __forceinline__ float tile_exp_all(uint32_t (&a)[128], float c, float bias, int lim,
-                                              uint64_t* tok, bool release) {
-  const uint64_t c2 = pk2(c, c), b2 = pk2(bias, bias);
-  uint64_t sum2[4] = {0, 0, 0, 0};
-  tile_exp<VAR, MASKED, PREFILL, CLAMP, 0, R>(a, c2, b2, lim, sum2);
-  if (release) {
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(tok);
-  }
-  tile_exp<VAR, MASKED, PREFILL, CLAMP, R, 128>(a, c2, b2, lim, sum2);
   const float2 s = up2(add2(add2(sum2[0], sum2[1]), add2(sum2[2], sum2[3])));
   return s.x + s.y;
-}
-
-template <int VAR, bool PREFILL>
-__device__ __forceinline__ float tile_exp_dispatch(uint32_t (&a)[128], float c, float bias, int lim,
-                                                   bool masked, bool clamp, uint64_t* tok, bool release) {
-  constexpr int R = Turns<VAR>::release;
-  if (PolyMask<VAR>::bits == 0)  // the clamp only guards the polynomial
-    return masked ? tile_exp_all<VAR, true, PREFILL, false, R>(a, c, bias, lim, tok, release)
-                  : tile_exp_all<VAR, false, PREFILL, false, R>(a, c, bias, lim, tok, release);
-  if (masked)
-    return clamp ? tile_exp_all<VAR, true, PREFILL, true, R>(a, c, bias, lim, tok, release)
-                 : tile_exp_all<VAR, true, PREFILL, false, R>(a, c, bias, lim, tok, release);
-  return clamp ? tile_exp_all<VAR, false, PREFILL, true, R>(a, c, bias, lim, tok, release)
-               : tile_exp_all<VAR, false, PREFILL, false, R>(a, c, bias, lim, tok, release);
 }
 
 template <int D, int VAR, bool CAUSAL, bool PACKED>
@@ -394,9 +305,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* pv_done = a_full + 2 * PB;  // [2][PB] P~V_g complete              (MMA commit)
   uint64_t* o_ready = pv_done + 2 * PB; // [2] O_g ready for the next P~V      (128 correction threads)
   uint64_t* l_full = o_ready + 2;     // [LS][2] final l_g of an item          (128 softmax threads)
-  uint64_t* tok0 = l_full + 2 * LS;   // [4] tile 0 warp w ended its exponentials (1 lane)
-  uint64_t* tok1 = tok0 + 4;          // [4] tile 1 warp w ended its exponentials (1 lane)
-  uint64_t* mma_done = tok1 + 4;
+  uint64_t* mma_done = l_full + 2 * LS;
   uint64_t* pv_mma_done = mma_done + 1;
   // Parity waits are only sound if no waiter can fall two phases behind the
   // barrier.  Per tile g, with u counting the kv steps of tile g over all
@@ -429,9 +338,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   //               for pv_done(u-PB), which needs o_ready of a step of item
   //               i+1, which the correction arrives only after its epilogue
   //               of item i consumed that slot.
-  //   tok0/tok1   strict alternation: tile 0's event e waits for tile 1's
-  //               event e-1 and tile 1's event e for tile 0's event e (an
-  //               inactive tile still takes part), so neither runs ahead.
   //   bar_q, q_empty: one phase per item per buffer; a buffer is reloaded
   //               only after the last S of the item that used it.
   //   k/v full/empty: the usual ring, one consumer each.
@@ -463,10 +369,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&o_ready[g], 128);
       for (int sl = 0; sl < LS; ++sl) mbar_init(&l_full[sl * 2 + g], 128);
     }
-    for (int w = 0; w < 4; ++w) {
-      mbar_init(&tok0[w], 1);
-      mbar_init(&tok1[w], 1);
-    }
     mbar_init(mma_done, 1);
     mbar_init(pv_mma_done, 1);
     *s_abort = 0;
@@ -488,111 +390,65 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int r = wq * 32 + lane;
     const uint32_t tS = tmem + (static_cast<uint32_t>(wq * 32) << 16) + g * 128;
     const uint32_t sP_g = smem_u32(smem + C::OFF_P) + g * PB * C::P_TILE;
-    uint64_t* tok_wait = g == 0 ? &tok1[wq] : &tok0[wq];
-    uint64_t* tok_mine = g == 0 ? &tok0[wq] : &tok1[wq];
-    // a score span that cannot reach 2^-124: |acc| <= 127^2 * D
-    constexpr float kSpan = 127.f * 127.f * D;
     if (C::PS) {
-      if (C::PREFILL) {
-        const uint32_t mg = kMagicBits;
-#pragma unroll
-        for (int cb = 0; cb < 16; ++cb) SAGE_TMEM_ST8_FILL(tS + cb * 8, mg);
-        tmem_wait_st();
-      }
       tc_fence_before();
       mbar_arrive(&s_free[g]);  // phase 0: the first S_g may be issued
     }
-    uint32_t u = 0, ul = 0, ev = 0;  // kv steps of tile g, items with tile g, token events
+    uint32_t u = 0, ul = 0;  // kv steps of tile g, items with tile g
     bool ok = true;
     for (int rd = 0; ok; ++rd) {
       const int item = item_of_round(p, rd);
       if (item < 0) break;
       const Item it = make_item<CAUSAL, PACKED>(p, item);
       if (PACKED && it.nkv == 0) continue;  // past the end of a short packed sequence
-      const bool act = g == 0 || it.has1;
+      if (g == 1 && !it.has1) continue;
       const int nkv_g = g == 0 ? it.nkv0 : it.nkv1;
       const int qb = it.qb0 + g;
-      float dq_l2e = 0.f, dk_next = 0.f, m = -INFINITY, l = 0.f;
+      const float dq_l2e = __fmul_rn(p.dq[static_cast<size_t>(it.bh) * p.nqb + qb], kLog2e);
       const float* dkp = p.dk + static_cast<size_t>(it.zkv) * p.nkvb;
-      if (act) {
-        dq_l2e = __fmul_rn(p.dq[static_cast<size_t>(it.bh) * p.nqb + qb], kLog2e);
-        dk_next = dkp[0];
-      }
-      // with turn-taking every warp steps through all kv steps of the item
-      // (an inactive tile still takes its turns); without, only its own
-      const int nsteps = Turns<VAR>::on ? it.nkv : (act ? nkv_g : 0);
-      for (int j = 0; j < nsteps; ++j, ++ev) {
-        const bool real = !Turns<VAR>::on || (act && j < nkv_g);
-        uint32_t a[128];
-        float c = 0.f, alpha = 0.f, bias = 0.f, m_new = 0.f;
-        int lim = kBN;
-        bool masked = false, clamp = false;
-        if (real) {
-          c = __fmul_rn(dq_l2e, dk_next);
-          if (j + 1 < nkv_g) dk_next = dkp[j + 1];
-          // tcgen05.ld/st below are warp-collective: every lane takes the same branch
-          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[g], u & 1, s_abort, tlim, 8))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          SAGE_TMEM_LD32(tS + 0, a);
-          SAGE_TMEM_LD32(tS + 32, (a + 32));
-          SAGE_TMEM_LD32(tS + 64, (a + 64));
-          SAGE_TMEM_LD32(tS + 96, (a + 96));
-          tmem_wait_ld();
-          if (C::PS) {  // S_g's columns may now take S_g(u+1)
-            if (C::PREFILL) {
-              const uint32_t mg = kMagicBits;
-#pragma unroll
-              for (int cb = 0; cb < 16; ++cb) SAGE_TMEM_ST8_FILL(tS + cb * 8, mg);
-              tmem_wait_st();
-            }
-            tc_fence_before();
-            mbar_arrive(&s_free[g]);
-          }
-          const int valid = it.n - j * kBN;  // keys left in this tile
-          masked = (CAUSAL && j == qb) || valid < kBN;
-          lim = masked ? min(valid, (CAUSAL && j == qb) ? r + 1 : kBN) : kBN;
-          int imax = masked ? tile_rowmax<true>(a, lim) : tile_rowmax<false>(a, lim);
-          if (C::PREFILL) imax -= static_cast<int>(kMagicBits);
-          // |imax| <= d * 127^2 < 2^22: the int -> float conversion is exact.
-          m_new = fmaxf(m, __fmul_rn(static_cast<float>(imax), c));
-          alpha = ex2_approx(m - m_new);  // 0 on the first tile
-          // 8+8: P tile and alpha slot u % 2 are free once P~V_g(u-2) is
-          // done (it is issued after the correction consumed alpha(u-2)).
-          // B: S_g(u) was issued after P~V_g(u-1), so both already hold.
-          if (C::PS && u >= PB &&
-              !__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[g * PB + u % PB], ((u - PB) / PB) & 1, s_abort,
-                                                 tlim, 15))) {
-            ok = false;
-            break;
-          }
-          // the correction warps rescale O_g while this thread computes P~
-          // (at an item's first step alpha is 0 and unused: the hand-off
-          // keeps one phase per step)
-          s_alpha[(g * PB + u % PB) * 128 + r] = alpha;
-          mbar_arrive(&a_full[g * PB + u % PB]);
-          bias = (VAR == 1) ? (p.log2_pr - m_new) : -m_new;
-          // every exponent acc*c + bias is >= -124 unless kSpan*c + m_new > 124
-          // (only the FMA-pipe exponentials need the bound)
-          if (PolyMask<VAR>::bits != 0) clamp = __any_sync(0xFFFFFFFFu, __fmaf_rn(kSpan, c, m_new) > 124.f);
-        }
-        // take the exp2 unit of this sub-partition: tile 0's event e follows
-        // tile 1's event e-1, tile 1's event e follows tile 0's event e
-        if (Turns<VAR>::on && (g == 1 || ev > 0) &&
-            !__all_sync(0xFFFFFFFFu, mbar_wait(tok_wait, g == 0 ? ((ev - 1) & 1) : (ev & 1), s_abort,
-                                               tlim, 16))) {
+      float dk_next = dkp[0], m = -INFINITY, l = 0.f;
+      for (int j = 0; j < nkv_g; ++j) {
+        const float c = __fmul_rn(dq_l2e, dk_next);
+        if (j + 1 < nkv_g) dk_next = dkp[j + 1];
+        // tcgen05.ld/st below are warp-collective: every lane takes the same branch
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&s_full[g], u & 1, s_abort, tlim, 8))) {
           ok = false;
           break;
         }
-        float rs = 0.f;
-        if (real) rs = tile_exp_dispatch<VAR, C::PREFILL>(a, c, bias, lim, masked, clamp, tok_mine, Turns<VAR>::on);
-        else if (Turns<VAR>::on) {  // an inactive tile still takes its turn
-          __syncwarp();
-          if (lane == 0) mbar_arrive(tok_mine);
+        tc_fence_after();
+        uint32_t a[128];
+        SAGE_TMEM_LD32(tS + 0, a);
+        SAGE_TMEM_LD32(tS + 32, (a + 32));
+        SAGE_TMEM_LD32(tS + 64, (a + 64));
+        SAGE_TMEM_LD32(tS + 96, (a + 96));
+        tmem_wait_ld();
+        if (C::PS) {  // S_g's columns may now take S_g(u+1)
+          tc_fence_before();
+          mbar_arrive(&s_free[g]);
         }
-        if (!real) continue;
+        const int valid = it.n - j * kBN;  // keys left in this tile
+        const bool masked = (CAUSAL && j == qb) || valid < kBN;
+        const int lim = masked ? min(valid, (CAUSAL && j == qb) ? r + 1 : kBN) : kBN;
+        const int imax = masked ? tile_rowmax<true>(a, lim) : tile_rowmax<false>(a, lim);
+        // |imax| <= d * 127^2 < 2^22: the int -> float conversion is exact.
+        const float m_new = fmaxf(m, __fmul_rn(static_cast<float>(imax), c));
+        const float alpha = ex2_approx(m - m_new);  // 0 on the first tile
+        // 8+8: the P tile and the alpha slot of buffer u % PB are free once
+        // P~V_g(u-PB) is done (it is issued after the correction consumed
+        // alpha(u-PB)).  B: S_g(u) ran after P~V_g(u-1), so both already hold.
+        if (C::PS && u >= PB &&
+            !__all_sync(0xFFFFFFFFu, mbar_wait(&pv_done[g * PB + u % PB], ((u - PB) / PB) & 1, s_abort,
+                                               tlim, 15))) {
+          ok = false;
+          break;
+        }
+        // the correction warps rescale O_g while this thread computes P~
+        // (at an item's first step alpha is 0 and unused: the hand-off keeps
+        // one phase per step)
+        s_alpha[(g * PB + u % PB) * 128 + r] = alpha;
+        mbar_arrive(&a_full[g * PB + u % PB]);
+        const float bias = (VAR == 1) ? (p.log2_pr - m_new) : -m_new;
+        const float rs = masked ? tile_exp<VAR, true>(a, c, bias, lim) : tile_exp<VAR, false>(a, c, bias, lim);
         l = __fmaf_rn(alpha, l, rs);
         if (C::PS) {
           // row r, 16-byte chunk k (keys 16k..16k+15) at the 128-byte-swizzled
@@ -611,13 +467,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(&p_full[g * PB + u % PB]);
         m = m_new;
         ++u;
-        if (j == nkv_g - 1) {
-          const int slot = static_cast<int>(ul % LS);
-          s_l[(slot * 2 + g) * 128 + r] = l;
-          mbar_arrive(&l_full[slot * 2 + g]);
-          ++ul;
-        }
       }
+      if (!ok) break;
+      const int slot = static_cast<int>(ul % LS);
+      s_l[(slot * 2 + g) * 128 + r] = l;
+      mbar_arrive(&l_full[slot * 2 + g]);
+      ++ul;
     }
   } else if (warp < 12) {
     // ---------------------------------------------------------------- correction + epilogue
@@ -821,7 +676,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk)
               mma_i8_ss(tmem + g * 128, ad + kk * 2, bd + kk * 2, C::IDESC_QK,
-                        (C::PREFILL || kk > 0) ? 1u : 0u);
+                        kk > 0 ? 1u : 0u);
             tc_commit(&s_full[g]);
             ++u[g];
           }

@@ -234,14 +234,6 @@ enum : uint32_t { AF_F16 = 0, AF_E4M3 = 0, AF_S8 = 1 };
       "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),       \
       "r"(r[29]), "r"(r[30]), "r"(r[31]))
 
-// 32 lanes x 8 columns of 32-bit tensor memory <- one value per lane (the
-// source of tcgen05.st is a block of consecutive registers: a narrow fill
-// keeps that block small).
-#define SAGE_TMEM_ST8_FILL(taddr, v)                                                   \
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"( \
-                   taddr),                                                             \
-               "r"(v))
-
 #define SAGE_TMEM_ST8(taddr, r)                                                         \
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"( \
                    taddr),                                                              \
