@@ -57,6 +57,9 @@ NCU_TRAFFIC = {
     ("ddd20728e76bed3c", "video_dit_h24_n32768_d128", "8+8"): 480.8e6,
     # 639.6 MB on the same small case (S issuer on warp 15)
     ("af2d12c4d8fbaca1", "video_dit_h24_n32768_d128", "8+8"): 479.7e6,
+    # 638.5 MB on the same small case: persistent scheduler, one CTA per item
+    # for long non-causal shapes
+    ("961ce71c0f592454", "video_dit_h24_n32768_d128", "8+8"): 478.9e6,
 }
 
 

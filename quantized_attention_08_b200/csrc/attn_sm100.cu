@@ -467,12 +467,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(&p_full[g * PB + u % PB]);
         m = m_new;
         ++u;
+        if (j == nkv_g - 1) {
+          const int slot = static_cast<int>(ul % LS);
+          s_l[(slot * 2 + g) * 128 + r] = l;
+          mbar_arrive(&l_full[slot * 2 + g]);
+          ++ul;
+        }
       }
-      if (!ok) break;
-      const int slot = static_cast<int>(ul % LS);
-      s_l[(slot * 2 + g) * 128 + r] = l;
-      mbar_arrive(&l_full[slot * 2 + g]);
-      ++ul;
     }
   } else if (warp < 12) {
     // ---------------------------------------------------------------- correction + epilogue
