@@ -252,10 +252,16 @@ __device__ __forceinline__ float tile_exp(uint32_t (&a)[128], float c, float bia
     float p[4];
 #pragma unroll
     for (int e = 0; e < 4; e += 2) {
-      // kMagicBits + acc reads as the fp32 value 1.5 * 2^23 + acc: one
-      // subtraction gives acc exactly
-      const uint64_t f2 = add2(pk2(__uint_as_float(a[i + e] + kMagicBits), __uint_as_float(a[i + e + 1] + kMagicBits)),
-                               magic2);
+      // acc as fp32, exactly (|acc| < 2^22).  8+8: a plain conversion;
+      // variant B: kMagicBits + acc reads as the fp32 value 1.5 * 2^23 + acc
+      // and one subtraction gives acc (each form measured faster in its
+      // variant's loop)
+      uint64_t f2;
+      if (VAR == 1) {
+        f2 = pk2(static_cast<float>(static_cast<int>(a[i + e])), static_cast<float>(static_cast<int>(a[i + e + 1])));
+      } else {
+        f2 = add2(pk2(__uint_as_float(a[i + e] + kMagicBits), __uint_as_float(a[i + e + 1] + kMagicBits)), magic2);
+      }
       const float2 x = up2(fma2(f2, c2, b2));
       p[e] = ex2_approx(x.x);
       p[e + 1] = ex2_approx(x.y);
