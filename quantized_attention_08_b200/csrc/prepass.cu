@@ -17,14 +17,21 @@
 //                delta_v = fp32(colmax) / v_r.
 //   k_quant    : one CTA per 128-token block of one head, for Q, K and V:
 //                block absmax -> delta -> codes.
-// With rotary tables, k_colstats and k_quant first rotate each fp16 row of K
-// (and Q) in registers ([SA1] implementation detail 1: RoPE and the
-// quantization in one pass, no rotated copy in HBM).
+// With rotary tables, k_colstats_rope and k_quant_rope rotate each fp16 row
+// of K (and Q) in registers first ([SA1] implementation detail 1: RoPE and
+// the quantization in one pass, no rotated copy in HBM).  Their threads own
+// both channels of every rotation pair (no shuffles), and one CTA serves
+// several heads of the same tokens, so that each slice of the cos / sin
+// tables is read once per head group rather than once per head.
 // Every value is bit-identical to the definition whatever the grid, because
 // the reductions are exact (integer sums, max) and each element's
 // arithmetic is a fixed sequence of correctly rounded fp32 operations.
 #include <cuda_fp16.h>
 #include <stdint.h>
+
+#include <algorithm>
+#include <atomic>
+#include <type_traits>
 
 #include "quant_div.h"
 #include "sage_internal.h"
@@ -54,65 +61,15 @@ __device__ __forceinline__ float4 ld_f4(const float* p) {
   return *reinterpret_cast<const float4*>(p);
 }
 
-// Rotary embedding of the 8 fp16 channels this thread holds at token t
-// (rotate-half pairing: channel i < D/2 pairs with i + D/2).  The partner
-// channels sit in lane ^ (TPR/2) of the same warp; the two partners load the
-// cos and the sin of their common 8 frequencies respectively and swap them.
-//   lower half: y = fl(fl(x*c) - fl(x'*s)),  upper half: y = fl(fl(x*c) + fl(x'*s)),
-// rounded to fp16.  t < 0 (a row past the end) yields zeros.  Every lane of
-// the warp must call this (shuffles).
-template <int D>
-__device__ __forceinline__ uint4 rope8(uint4 x, int t, int cg, const float* __restrict__ cosT,
-                                       const float* __restrict__ sinT) {
-  constexpr int TPR = D / 8, H2 = D / 2;
-  const bool upper = cg >= TPR / 2;
-  uint4 xp;
-  xp.x = __shfl_xor_sync(0xFFFFFFFFu, x.x, TPR / 2);
-  xp.y = __shfl_xor_sync(0xFFFFFFFFu, x.y, TPR / 2);
-  xp.z = __shfl_xor_sync(0xFFFFFFFFu, x.z, TPR / 2);
-  xp.w = __shfl_xor_sync(0xFFFFFFFFu, x.w, TPR / 2);
-  const float* tab = (upper ? sinT : cosT) + static_cast<size_t>(t < 0 ? 0 : t) * H2 + (cg % (TPR / 2)) * 8;
-  float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
-  if (t >= 0) {
-    a0 = ld_f4(tab);
-    a1 = ld_f4(tab + 4);
-  }
-  float4 b0, b1;
-  b0.x = __shfl_xor_sync(0xFFFFFFFFu, a0.x, TPR / 2);
-  b0.y = __shfl_xor_sync(0xFFFFFFFFu, a0.y, TPR / 2);
-  b0.z = __shfl_xor_sync(0xFFFFFFFFu, a0.z, TPR / 2);
-  b0.w = __shfl_xor_sync(0xFFFFFFFFu, a0.w, TPR / 2);
-  b1.x = __shfl_xor_sync(0xFFFFFFFFu, a1.x, TPR / 2);
-  b1.y = __shfl_xor_sync(0xFFFFFFFFu, a1.y, TPR / 2);
-  b1.z = __shfl_xor_sync(0xFFFFFFFFu, a1.z, TPR / 2);
-  b1.w = __shfl_xor_sync(0xFFFFFFFFu, a1.w, TPR / 2);
-  const float ta[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-  const float tb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-  const uint32_t w[4] = {x.x, x.y, x.z, x.w}, wp[4] = {xp.x, xp.y, xp.z, xp.w};
-  uint32_t out[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
-    const float2 g = __half22float2(*reinterpret_cast<const __half2*>(&wp[e]));
-    const float c0 = upper ? tb[2 * e] : ta[2 * e], s0 = upper ? ta[2 * e] : tb[2 * e];
-    const float c1 = upper ? tb[2 * e + 1] : ta[2 * e + 1], s1 = upper ? ta[2 * e + 1] : tb[2 * e + 1];
-    const float y0 = upper ? __fadd_rn(__fmul_rn(f.x, c0), __fmul_rn(g.x, s0))
-                           : __fsub_rn(__fmul_rn(f.x, c0), __fmul_rn(g.x, s0));
-    const float y1 = upper ? __fadd_rn(__fmul_rn(f.y, c1), __fmul_rn(g.y, s1))
-                           : __fsub_rn(__fmul_rn(f.y, c1), __fmul_rn(g.y, s1));
-    const __half2 h = __floats2half2_rn(y0, y1);
-    out[e] = *reinterpret_cast<const uint32_t*>(&h);
-  }
-  return make_uint4(out[0], out[1], out[2], out[3]);
-}
+// Heads per CTA of the rotary kernels: the largest of 4, 2, 1 dividing the
+// slab count per batch entry (so that a CTA's heads share their tokens).
+inline int rope_group(int heads) { return heads % 4 == 0 ? 4 : heads % 2 == 0 ? 2 : 1; }
 
-template <int D, bool ROPE>
+template <int D>
 __global__ void __launch_bounds__(kThreads) k_colstats(const uint4* __restrict__ k,
                                                        const uint4* __restrict__ v, SeqLayout seq,
                                                        int Hkv, int nchunk, long long* __restrict__ ksum,
-                                                       uint32_t* __restrict__ vmax,
-                                                       const float* __restrict__ cosT,
-                                                       const float* __restrict__ sinT) {
+                                                       uint32_t* __restrict__ vmax) {
   constexpr int TPR = D / 8;             // threads per row: one uint4 (8 halves) each
   constexpr int RPI = kThreads / TPR;    // rows per iteration
   const int chunk = blockIdx.x, slab = blockIdx.y;
@@ -133,8 +90,7 @@ __global__ void __launch_bounds__(kThreads) k_colstats(const uint4* __restrict__
   // 16-byte loads per array are in flight; rows past the chunk read as +0,
   // which adds nothing to either statistic.
   constexpr int kUnroll = 4;
-  // (all lanes of a warp run the same iterations: the rotary path shuffles)
-  for (int r = r0 + rl, rw = r0 + (rl & ~(32 / TPR - 1)); rw < r1; r += kUnroll * RPI, rw += kUnroll * RPI) {
+  for (int r = r0 + rl; r < r1; r += kUnroll * RPI) {
     uint4 xk[kUnroll], xv[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -142,13 +98,6 @@ __global__ void __launch_bounds__(kThreads) k_colstats(const uint4* __restrict__
       const bool in = rr < r1;
       xk[u] = (k != nullptr && in) ? ld_stream(k + base + static_cast<size_t>(rr) * TPR) : make_uint4(0, 0, 0, 0);
       xv[u] = (v != nullptr && in) ? ld_stream(v + base + static_cast<size_t>(rr) * TPR) : make_uint4(0, 0, 0, 0);
-    }
-    if (ROPE && k != nullptr) {
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int rr = r + u * RPI;
-        xk[u] = rope8<D>(xk[u], rr < r1 ? rr : -1, cg, cosT, sinT);
-      }
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -188,6 +137,167 @@ __global__ void __launch_bounds__(kThreads) k_colstats(const uint4* __restrict__
     const size_t o = (static_cast<size_t>(slab) * nchunk + chunk) * D + c;
     if (k != nullptr) ksum[o] = __double2ll_rn(__dmul_rn(s, 0x1p24));  // an integer: exact
     if (v != nullptr) vmax[o] = mx;
+  }
+}
+
+// ---------------------------------------------------------------- fp32 pairs
+// Lane-wise IEEE fp32 operations on two values (each lane rounded to nearest
+// even, exactly as the scalar operation), two per instruction.  A product
+// must not feed f2_add / f2_sub directly (see rope2).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// the two fp16 values of w as fp32 (exact)
+__device__ __forceinline__ uint64_t f2_from_h2(uint32_t w) {
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+  return f2_pack(f.x, f.y);
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+// int8 codes of four x values (two lanes each), delta > 0, r = RN(1/delta),
+// nd = -delta: code = RN(x / delta) (div_rn_nosign of quant_div.h, lane-wise:
+// the remainder fma(q, -delta, x) is the same exact value as fma(-q, delta,
+// x)), rounded to an integer by the 1.5 * 2^23 add of rne_code8; bytes in
+// lane order.
+__device__ __forceinline__ uint32_t codes4(uint64_t x01, uint64_t x23, uint64_t nd2, uint64_t r2) {
+  const uint64_t magic2 = f2_pack(12582912.f, 12582912.f);
+  const uint64_t q01 = f2_mul(x01, r2), q23 = f2_mul(x23, r2);
+  const uint64_t y01 = f2_fma(f2_fma(q01, nd2, x01), r2, q01);
+  const uint64_t y23 = f2_fma(f2_fma(q23, nd2, x23), r2, q23);
+  const uint64_t c01 = f2_add(y01, magic2), c23 = f2_add(y23, magic2);
+  const uint32_t lo = prmt(static_cast<uint32_t>(c01), static_cast<uint32_t>(c01 >> 32), 0x0040u);
+  const uint32_t hi = prmt(static_cast<uint32_t>(c23), static_cast<uint32_t>(c23 >> 32), 0x0040u);
+  return prmt(lo, hi, 0x5410u);
+}
+
+// Rotary embedding, rotate-half pairing (channel i < D/2 pairs with
+// i + D/2), of two channel pairs at once: wl holds fp16 x_i, x_i+1 of the
+// lower half, wh their partners y, c / s the cos and sin of the two
+// frequencies: lower y = fl(fl(x c) - fl(y s)), upper fl(fl(y c) + fl(x s)),
+// each then rounded to fp16.
+// The products are paired; the sums are scalar: ptxas contracts a paired
+// product that feeds a paired add or sub into a fused multiply-add whatever
+// the rounding qualifiers (and -fmad=false), which would round once instead
+// of twice; scalar .rn adds are never contracted.
+__device__ __forceinline__ void rope2(uint32_t& wl, uint32_t& wh, uint64_t c2, uint64_t s2) {
+  const uint64_t x = f2_from_h2(wl), y = f2_from_h2(wh);
+  const float2 xc = f2_unpack(f2_mul(x, c2)), ys = f2_unpack(f2_mul(y, s2));
+  const float2 yc = f2_unpack(f2_mul(y, c2)), xs = f2_unpack(f2_mul(x, s2));
+  const __half2 rl = __floats2half2_rn(__fsub_rn(xc.x, ys.x), __fsub_rn(xc.y, ys.y));
+  const __half2 rh = __floats2half2_rn(__fadd_rn(yc.x, xs.x), __fadd_rn(yc.y, xs.y));
+  wl = *reinterpret_cast<const uint32_t*>(&rl);
+  wh = *reinterpret_cast<const uint32_t*>(&rh);
+}
+
+// K column sums with rotary embedding: one CTA per (256-token chunk, G
+// consecutive heads of one batch entry).  Rows outer, heads inner: a thread
+// loads the cos / sin of its 8 frequencies at a token once and rotates that
+// token's row in each of the G heads.  Sums are exact (see k_colstats), so
+// their order is free.
+template <int D, int G>
+__global__ void __launch_bounds__(kThreads, 2) k_colstats_rope(const uint4* __restrict__ k, SeqLayout seq,
+                                                               int Hkv, int nchunk,
+                                                               long long* __restrict__ ksum,
+                                                               const float* __restrict__ cosT,
+                                                               const float* __restrict__ sinT) {
+  constexpr int TPR = D / 8, TP = TPR / 2, H2 = D / 2;
+  constexpr int RPI = kThreads / TP;  // rows per iteration
+  const int chunk = blockIdx.x, z0 = blockIdx.y * G;
+  const int j = threadIdx.x % TP, rl = threadIdx.x / TP;
+  size_t row0[G];
+  int N = 0;
+#pragma unroll
+  for (int h = 0; h < G; ++h) slab_rows(seq, z0 + h, Hkv, &row0[h], &N);  // same N for the group
+  const int r0 = chunk * kStatRows, r1 = min(N, r0 + kStatRows);
+  if (r0 >= N) return;  // a chunk past the end of a short sequence
+
+  double acc[G][16];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[h][e] = 0.0;
+#pragma unroll 1
+  for (int r = r0 + rl; r < r1; r += RPI) {
+    const float* ct = cosT + static_cast<size_t>(r) * H2 + 8 * j;
+    const float* st = sinT + static_cast<size_t>(r) * H2 + 8 * j;
+    const float4 c0 = ld_f4(ct), c1 = ld_f4(ct + 4), s0 = ld_f4(st), s1 = ld_f4(st + 4);
+    uint4 lo[G], hi[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const uint4* row = k + (row0[h] + r) * TPR;
+      lo[h] = ld_stream(row + j);
+      hi[h] = ld_stream(row + j + TP);
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      rope2(lo[h].x, hi[h].x, f2_pack(c0.x, c0.y), f2_pack(s0.x, s0.y));
+      rope2(lo[h].y, hi[h].y, f2_pack(c0.z, c0.w), f2_pack(s0.z, s0.w));
+      rope2(lo[h].z, hi[h].z, f2_pack(c1.x, c1.y), f2_pack(s1.x, s1.y));
+      rope2(lo[h].w, hi[h].w, f2_pack(c1.z, c1.w), f2_pack(s1.z, s1.w));
+      const uint32_t wl[4] = {lo[h].x, lo[h].y, lo[h].z, lo[h].w}, wh[4] = {hi[h].x, hi[h].y, hi[h].z, hi[h].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        add_f16x2(acc[h][2 * e], acc[h][2 * e + 1], wl[e]);
+        add_f16x2(acc[h][8 + 2 * e], acc[h][8 + 2 * e + 1], wh[e]);
+      }
+    }
+  }
+  // lanes of a warp with the same j hold the same channels: fold them, then
+  // the warps through shared memory
+#pragma unroll
+  for (int o = TP; o < 32; o <<= 1)
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < 16; ++e) acc[h][e] = __dadd_rn(acc[h][e], __shfl_xor_sync(0xFFFFFFFFu, acc[h][e], o));
+  __shared__ double s_sum[kThreads / 32][G][D];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane < TP) {
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        s_sum[w][h][8 * j + e] = acc[h][e];
+        s_sum[w][h][H2 + 8 * j + e] = acc[h][8 + e];
+      }
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < G * D; t += kThreads) {
+    const int h = t / D, c = t % D;
+    double sum = 0.0;
+#pragma unroll
+    for (int i = 0; i < kThreads / 32; ++i) sum = __dadd_rn(sum, s_sum[i][h][c]);
+    ksum[(static_cast<size_t>(z0 + h) * nchunk + chunk) * D + c] = __double2ll_rn(__dmul_rn(sum, 0x1p24));
   }
 }
 
@@ -263,8 +373,8 @@ struct QuantJobs {
   int n_q, n_k, n_v;    // number of (slab, block) jobs of each kind
 };
 
-template <int D, bool ROPE>
-__global__ void __launch_bounds__(kThreads, ROPE ? 3 : 4) k_quant(const QuantJobs J) {
+template <int D>
+__global__ void __launch_bounds__(kThreads, 4) k_quant(const QuantJobs J) {
   constexpr int TPR = D / 8;                  // uint4 per token row
   constexpr int U = 128 * TPR / kThreads;     // uint4 per thread
   __shared__ float s_red[kThreads / 32];
@@ -296,13 +406,6 @@ __global__ void __launch_bounds__(kThreads, ROPE ? 3 : 4) k_quant(const QuantJob
   for (int u = 0; u < U; ++u) {
     const int idx = threadIdx.x + kThreads * u;
     raw[u] = (idx / TPR < rows) ? ld_stream(src + idx) : make_uint4(0, 0, 0, 0);
-  }
-  if (ROPE && kind != 2) {  // kind is uniform over the CTA
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int idx = threadIdx.x + kThreads * u;
-      raw[u] = rope8<D>(raw[u], idx / TPR < rows ? blk * 128 + idx / TPR : -1, cg, J.cos_t, J.sin_t);
-    }
   }
 
   if (kind == 2) {
@@ -387,6 +490,173 @@ __global__ void __launch_bounds__(kThreads, ROPE ? 3 : 4) k_quant(const QuantJob
   }
 }
 
+// Q and K blocks with rotary embedding: one CTA per (128-token block, G
+// consecutive heads of one batch entry, Q or K); jobs [0, n_q) are Q
+// groups, [n_q, n_q + n_k) K groups.  The block's cos / sin rows are staged
+// once in shared memory, then each head's block is rotated and quantized
+// with the values of k_quant: x = fp32(q) * sm_scale or fp32(k) - mean_k,
+// delta = RN(absmax / 127), codes RN(x / delta).  A thread holds channel
+// groups j and j + TP (both halves of its rotation pairs) of rows
+// rl + u * RPP.  The block absmax is taken on the rotated fp16 values: fp32
+// rounding is monotonic, so max |fl(f s)| = fl(max |f| * s) and, per
+// channel, max |fl(f - m)| = max(|fl(max f - m)|, |fl(min f - m)|).
+template <int D>
+constexpr int rope_tab_bytes() { return 128 * D * 4; }  // cos and sin, D/2 each, of 128 tokens
+
+template <int D, int G>
+__global__ void __launch_bounds__(kThreads, 3) k_quant_rope(const QuantJobs J) {
+  constexpr int TPR = D / 8, TP = TPR / 2, H2 = D / 2;
+  constexpr int RPP = kThreads / TP;  // rows per pass
+  constexpr int R = 128 / RPP;        // rows per thread
+  // [token][quarter][j] float4; quarters: cos of frequencies 8j..8j+3,
+  // cos of 8j+4..8j+7, then the same of sin (lanes j read adjacent 16 bytes)
+  extern __shared__ float4 s_tab[];
+  __shared__ float s_red[2][kThreads / 32];
+
+  int job = blockIdx.x;
+  const int kind = job < J.n_q ? 0 : 1;
+  if (kind == 1) job -= J.n_q;
+  const int Hs = kind == 0 ? J.H : J.Hkv;
+  const int z0 = (job / J.nb) * G, blk = job % J.nb;
+  size_t srow;
+  int len;
+  slab_rows(J.seq, z0, Hs, &srow, &len);  // the same tokens for all G heads
+  const int rows = min(128, len - blk * 128);
+  if (rows <= 0) return;  // a block past the end of a short sequence
+  // head z0 + h starts T rows after head z0 + h - 1 (both layouts)
+  const size_t row_b = srow + static_cast<size_t>(blk) * 128;
+  const uint4* src0 = (kind == 0 ? J.q : J.k) + row_b * TPR;
+  uint2* dst0 = (kind == 0 ? J.q_hat : J.k_hat) + row_b * TPR;
+  const size_t hstride = static_cast<size_t>(J.seq.T) * TPR;
+  float* dlt = (kind == 0 ? J.delta_q : J.delta_k) + static_cast<size_t>(z0) * J.nb + blk;
+  const int j = threadIdx.x % TP, rl = threadIdx.x / TP;
+
+  // FULL: all 128 rows present (no per-row predicates)
+  auto run = [&](auto full_tag) {
+    constexpr bool FULL = decltype(full_tag)::value;
+    uint4 lo[R], hi[R];
+    auto load_block = [&](int h) {
+      const uint4* src = src0 + h * hstride;
+#pragma unroll
+      for (int u = 0; u < R; ++u) {
+        const int row = rl + u * RPP;
+        const bool in = FULL || row < rows;
+        lo[u] = in ? ld_stream(src + row * TPR + j) : make_uint4(0, 0, 0, 0);
+        hi[u] = in ? ld_stream(src + row * TPR + j + TP) : make_uint4(0, 0, 0, 0);
+      }
+    };
+    load_block(0);  // in flight while the table is staged
+    {
+      const float* tabs[2] = {J.cos_t + static_cast<size_t>(blk) * 128 * H2,
+                              J.sin_t + static_cast<size_t>(blk) * 128 * H2};
+#pragma unroll 2
+      for (int i = threadIdx.x; i < 2 * 128 * (H2 / 4); i += kThreads) {
+        const int tab = i / (128 * (H2 / 4)), row = (i / (H2 / 4)) % 128, f4 = i % (H2 / 4);
+        if (FULL || row < rows)
+          s_tab[(row * 4 + tab * 2 + (f4 & 1)) * TP + (f4 >> 1)] = ld_f4(tabs[tab] + row * H2 + 4 * f4);
+      }
+    }
+    __syncthreads();
+
+    for (int h = 0; h < G; ++h) {
+      if (h > 0) load_block(h);
+#pragma unroll
+      for (int u = 0; u < R; ++u) {
+        const int row = rl + u * RPP;
+        if (FULL || row < rows) {  // table rows past the end are not staged
+          const float4* t = s_tab + row * 4 * TP + j;
+          const float4 c0 = t[0], c1 = t[TP], s0 = t[2 * TP], s1 = t[3 * TP];
+          rope2(lo[u].x, hi[u].x, f2_pack(c0.x, c0.y), f2_pack(s0.x, s0.y));
+          rope2(lo[u].y, hi[u].y, f2_pack(c0.z, c0.w), f2_pack(s0.z, s0.w));
+          rope2(lo[u].z, hi[u].z, f2_pack(c1.x, c1.y), f2_pack(s1.x, s1.y));
+          rope2(lo[u].w, hi[u].w, f2_pack(c1.z, c1.w), f2_pack(s1.z, s1.w));
+        }
+      }
+      // this thread's share of the block absmax
+      float amax = 0.f;
+      uint64_t m2[8];  // K: mean_k of channels 8j.. (m2[0..3]) and H2+8j.. (m2[4..7]), in pairs
+      if (kind == 0) {
+        uint32_t mag = 0;  // two fp16 magnitudes (rows past the end are +0)
+#pragma unroll
+        for (int u = 0; u < R; ++u) {
+          const uint32_t w[8] = {lo[u].x, lo[u].y, lo[u].z, lo[u].w, hi[u].x, hi[u].y, hi[u].z, hi[u].w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mag = __vmaxu2(mag, w[e] & 0x7FFF7FFFu);
+        }
+        const uint32_t mx = max(mag & 0xFFFFu, mag >> 16);
+        amax = __fmul_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(mx))), fabsf(J.sm_scale));
+      } else {
+        const float* mk = J.mean_k + static_cast<size_t>(z0 + h) * D;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          m2[e] = f2_pack(mk[8 * j + 2 * e], mk[8 * j + 2 * e + 1]);
+          m2[4 + e] = f2_pack(mk[H2 + 8 * j + 2 * e], mk[H2 + 8 * j + 2 * e + 1]);
+        }
+        if (FULL || rl < rows) {  // row rl (u = 0) is this thread's first; others may be past the end
+          __half2 cmax[8], cmin[8];
+          {
+            const uint32_t w[8] = {lo[0].x, lo[0].y, lo[0].z, lo[0].w, hi[0].x, hi[0].y, hi[0].z, hi[0].w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) cmax[e] = cmin[e] = *reinterpret_cast<const __half2*>(&w[e]);
+          }
+#pragma unroll
+          for (int u = 1; u < R; ++u) {
+            if (FULL || rl + u * RPP < rows) {
+              const uint32_t w[8] = {lo[u].x, lo[u].y, lo[u].z, lo[u].w, hi[u].x, hi[u].y, hi[u].z, hi[u].w};
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const __half2 v = *reinterpret_cast<const __half2*>(&w[e]);
+                cmax[e] = __hmax2(cmax[e], v);
+                cmin[e] = __hmin2(cmin[e], v);
+              }
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float2 a = f2_unpack(f2_sub(f2_from_h2(*reinterpret_cast<const uint32_t*>(&cmax[e])), m2[e]));
+            const float2 b = f2_unpack(f2_sub(f2_from_h2(*reinterpret_cast<const uint32_t*>(&cmin[e])), m2[e]));
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(b.x), fabsf(b.y))));
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      // one barrier per head: s_red alternates, and a warp writes slot h & 1
+      // again (head h + 2) only after every warp passed head h + 1's barrier,
+      // i.e. after it read head h's slot
+      if ((threadIdx.x & 31) == 0) s_red[h & 1][threadIdx.x >> 5] = amax;
+      __syncthreads();
+      amax = s_red[h & 1][0];
+#pragma unroll
+      for (int i = 1; i < kThreads / 32; ++i) amax = fmaxf(amax, s_red[h & 1][i]);
+      const float delta = __fdiv_rn(amax, 127.f);
+      if (threadIdx.x == 0) dlt[static_cast<size_t>(h) * J.nb] = delta;
+      const float r = delta != 0.f ? __frcp_rn(delta) : 0.f;
+      const uint64_t r2 = f2_pack(r, r), nd2 = f2_pack(-delta, -delta), s2 = f2_pack(J.sm_scale, J.sm_scale);
+      uint2* dst = dst0 + h * hstride;
+#pragma unroll
+      for (int u = 0; u < R; ++u) {
+        const int row = rl + u * RPP;
+        if (!FULL && row >= rows) continue;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const uint4 v = half ? hi[u] : lo[u];
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          uint64_t x[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            x[e] = kind == 0 ? f2_mul(f2_from_h2(w[e]), s2) : f2_sub(f2_from_h2(w[e]), m2[half * 4 + e]);
+          uint2 out = make_uint2(0u, 0u);
+          if (delta != 0.f) out = make_uint2(codes4(x[0], x[1], nd2, r2), codes4(x[2], x[3], nd2, r2));
+          dst[row * TPR + j + half * TP] = out;
+        }
+      }
+    }
+  };
+  if (rows == 128) run(std::true_type());
+  else run(std::false_type());
+}
+
 // ---------------------------------------------------------------- launchers
 size_t stat_chunks(int N) { return static_cast<size_t>((N + kStatRows - 1) / kStatRows); }
 
@@ -406,16 +676,26 @@ cudaError_t launch_colstats(const void* k, const void* v, int slabs, int N, int 
   seq = fixed_or(seq, N);
   const int nchunk = static_cast<int>(stat_chunks(seq.max_len));
   if (nchunk == 0 || slabs == 0) return cudaSuccess;
-  dim3 grid(nchunk, slabs);
   const uint4* k4 = static_cast<const uint4*>(k);
   const uint4* v4 = static_cast<const uint4*>(v);
-  const bool rope = cos_t != nullptr && k != nullptr;
-  if (D == 128) {
-    if (rope) k_colstats<128, true><<<grid, kThreads, 0, st>>>(k4, v4, seq, Hkv, nchunk, ksum, vmax, cos_t, sin_t);
-    else k_colstats<128, false><<<grid, kThreads, 0, st>>>(k4, v4, seq, Hkv, nchunk, ksum, vmax, nullptr, nullptr);
-  } else {
-    if (rope) k_colstats<64, true><<<grid, kThreads, 0, st>>>(k4, v4, seq, Hkv, nchunk, ksum, vmax, cos_t, sin_t);
-    else k_colstats<64, false><<<grid, kThreads, 0, st>>>(k4, v4, seq, Hkv, nchunk, ksum, vmax, nullptr, nullptr);
+  if (cos_t != nullptr && k != nullptr) {
+    // rotated K sums per head group; V maxima (if any) by the plain kernel
+    const int G = Hkv % 2 == 0 ? 2 : 1;
+    const dim3 grid(nchunk, slabs / G);
+    if (D == 128) {
+      if (G == 2) k_colstats_rope<128, 2><<<grid, kThreads, 0, st>>>(k4, seq, Hkv, nchunk, ksum, cos_t, sin_t);
+      else k_colstats_rope<128, 1><<<grid, kThreads, 0, st>>>(k4, seq, Hkv, nchunk, ksum, cos_t, sin_t);
+    } else {
+      if (G == 2) k_colstats_rope<64, 2><<<grid, kThreads, 0, st>>>(k4, seq, Hkv, nchunk, ksum, cos_t, sin_t);
+      else k_colstats_rope<64, 1><<<grid, kThreads, 0, st>>>(k4, seq, Hkv, nchunk, ksum, cos_t, sin_t);
+    }
+    k4 = nullptr;
+    ksum = nullptr;
+  }
+  if (k4 != nullptr || v4 != nullptr) {
+    const dim3 grid(nchunk, slabs);
+    if (D == 128) k_colstats<128><<<grid, kThreads, 0, st>>>(k4, v4, seq, Hkv, nchunk, ksum, vmax);
+    else k_colstats<64><<<grid, kThreads, 0, st>>>(k4, v4, seq, Hkv, nchunk, ksum, vmax);
   }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) set_error_detail("column statistics kernel launch", e);
@@ -432,6 +712,33 @@ cudaError_t launch_finalize(const long long* ksum, const uint32_t* vmax, int sla
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) set_error_detail("finalize kernel launch", e);
   return e;
+}
+
+// Opt-in to the rotary table's dynamic shared memory, once per device and
+// instantiation (the attribute is per device).
+template <int D, int G>
+static cudaError_t quant_rope_attr() {
+  constexpr int kMaxDev = 64;
+  static std::atomic<bool> done[kMaxDev];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(k_quant_rope<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, rope_tab_bytes<D>());
+  if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+  return e;
+}
+
+template <int D, int G>
+static cudaError_t launch_quant_rope(const QuantJobs& J, int total, cudaStream_t st) {
+  cudaError_t e = quant_rope_attr<D, G>();
+  if (e != cudaSuccess) {
+    set_error_detail("cudaFuncSetAttribute(rotary quantization)", e, rope_tab_bytes<D>());
+    return e;
+  }
+  k_quant_rope<D, G><<<total, kThreads, rope_tab_bytes<D>(), st>>>(J);
+  return cudaSuccess;
 }
 
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st) {
@@ -456,15 +763,31 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st) {
   J.n_q = a.q ? a.B * a.H * J.nb : 0;
   J.n_k = a.k ? a.B * a.H_kv * J.nb : 0;
   J.n_v = a.v ? a.B * a.H_kv * J.nb : 0;
+  if (J.n_q + J.n_k + J.n_v == 0) return cudaSuccess;
+  if (a.cos_t != nullptr && J.n_q + J.n_k > 0) {
+    // Q and K in head groups with the rotary table; V below on its own
+    const int G = std::min(rope_group(a.H), rope_group(a.H_kv));
+    QuantJobs R = J;
+    R.n_q = J.n_q / G;
+    R.n_k = J.n_k / G;
+    R.n_v = 0;
+    const int total = R.n_q + R.n_k;
+    cudaError_t e;
+    if (a.d == 128) {
+      e = G == 4 ? launch_quant_rope<128, 4>(R, total, st)
+                 : G == 2 ? launch_quant_rope<128, 2>(R, total, st) : launch_quant_rope<128, 1>(R, total, st);
+    } else {
+      e = G == 4 ? launch_quant_rope<64, 4>(R, total, st)
+                 : G == 2 ? launch_quant_rope<64, 2>(R, total, st) : launch_quant_rope<64, 1>(R, total, st);
+    }
+    if (e != cudaSuccess) return e;
+    J.n_q = 0;
+    J.n_k = 0;
+  }
   const int total = J.n_q + J.n_k + J.n_v;
-  if (total == 0) return cudaSuccess;
-  const bool rope = a.cos_t != nullptr;
-  if (a.d == 128) {
-    if (rope) k_quant<128, true><<<total, kThreads, 0, st>>>(J);
-    else k_quant<128, false><<<total, kThreads, 0, st>>>(J);
-  } else {
-    if (rope) k_quant<64, true><<<total, kThreads, 0, st>>>(J);
-    else k_quant<64, false><<<total, kThreads, 0, st>>>(J);
+  if (total > 0) {
+    if (a.d == 128) k_quant<128><<<total, kThreads, 0, st>>>(J);
+    else k_quant<64><<<total, kThreads, 0, st>>>(J);
   }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) set_error_detail("quantization kernel launch", e);

@@ -57,8 +57,10 @@ def check_rope_prepass(sage, q, k, v, sm_scale):
     return got, (qr, kr)
 
 
+# head groups of the rotary kernels: 2 (H 2 / 4, H_kv 2), 1 (H_kv 1 or 3),
+# 4 (H 8, H_kv 4; and H 16 below); ragged, one-token and multi-block lengths
 @pytest.mark.parametrize("shape", [(1, 2, 2, 256, 64), (2, 4, 2, 300, 128), (1, 3, 1, 77, 64),
-                                   (1, 2, 2, 1, 128)],
+                                   (1, 2, 2, 1, 128), (2, 6, 3, 130, 64), (1, 8, 4, 520, 128)],
                          ids=lambda s: "B{}_H{}_Hkv{}_N{}_d{}".format(*s))
 def test_rope_prepass_bit_exact_small(sage, shape):
     B, H, Hk, N, d = shape
