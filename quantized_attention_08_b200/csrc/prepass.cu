@@ -33,7 +33,6 @@
 #include <atomic>
 #include <type_traits>
 
-#include "quant_div.h"
 #include "sage_internal.h"
 
 namespace sage {
@@ -185,10 +184,13 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 // int8 codes of four x values (two lanes each), delta > 0, r = RN(1/delta),
-// nd = -delta: code = RN(x / delta) (div_rn_nosign of quant_div.h, lane-wise:
+// nd = -delta: y = RN(x / delta) (div_rn_nosign of quant_div.h, lane-wise:
 // the remainder fma(q, -delta, x) is the same exact value as fma(-q, delta,
-// x)), rounded to an integer by the 1.5 * 2^23 add of rne_code8; bytes in
-// lane order.
+// x)), then rounded half-even to an integer: adding 1.5 * 2^23 leaves it in
+// the low mantissa bits, whose low byte is the two's-complement code; bytes
+// in lane order.  No clamp is needed: |x| <= absmax and delta = RN(absmax /
+// 127) >= absmax / 127 * (1 - 2^-24), so |y| <= 127 * (1 + 2^-22) rounds to
+// at most 127; -0 and +0 both give code 0.
 __device__ __forceinline__ uint32_t codes4(uint64_t x01, uint64_t x23, uint64_t nd2, uint64_t r2) {
   const uint64_t magic2 = f2_pack(12582912.f, 12582912.f);
   const uint64_t q01 = f2_mul(x01, r2), q23 = f2_mul(x23, r2);
@@ -219,68 +221,109 @@ __device__ __forceinline__ void rope2(uint32_t& wl, uint32_t& wh, uint64_t c2, u
   wh = *reinterpret_cast<const uint32_t*>(&rh);
 }
 
-// K column sums with rotary embedding: one CTA per (256-token chunk, G
-// consecutive heads of one batch entry).  Rows outer, heads inner: a thread
-// loads the cos / sin of its 8 frequencies at a token once and rotates that
-// token's row in each of the G heads.  Sums are exact (see k_colstats), so
-// their order is free.
-template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 2) k_colstats_rope(const uint4* __restrict__ k, SeqLayout seq,
+// Column statistics with rotary embedding: one CTA per (256-token chunk, G
+// consecutive heads of one batch entry): exact sums of the rotated K and,
+// if v is given (then G = 1), the max |V| as in k_colstats.  Rows outer,
+// heads inner: a thread loads the cos / sin of its 8 frequencies at a
+// token once and rotates that token's row in each of the G heads; U rows
+// per thread are loaded before any is reduced.  Sums are exact (see
+// k_colstats), so their order is free.
+template <int D, int G, int U>
+__global__ void __launch_bounds__(kThreads, 2) k_colstats_rope(const uint4* __restrict__ k,
+                                                               const uint4* __restrict__ v, SeqLayout seq,
                                                                int Hkv, int nchunk,
                                                                long long* __restrict__ ksum,
+                                                               uint32_t* __restrict__ vmax,
                                                                const float* __restrict__ cosT,
                                                                const float* __restrict__ sinT) {
   constexpr int TPR = D / 8, TP = TPR / 2, H2 = D / 2;
   constexpr int RPI = kThreads / TP;  // rows per iteration
   const int chunk = blockIdx.x, z0 = blockIdx.y * G;
   const int j = threadIdx.x % TP, rl = threadIdx.x / TP;
-  size_t row0[G];
+  size_t row0;
   int N = 0;
-#pragma unroll
-  for (int h = 0; h < G; ++h) slab_rows(seq, z0 + h, Hkv, &row0[h], &N);  // same N for the group
+  slab_rows(seq, z0, Hkv, &row0, &N);  // head z0 + h starts h * T rows later (same tokens)
   const int r0 = chunk * kStatRows, r1 = min(N, r0 + kStatRows);
   if (r0 >= N) return;  // a chunk past the end of a short sequence
+  const size_t hstride = static_cast<size_t>(seq.T) * TPR;
+  const uint4* kb = k + row0 * TPR + j;
+  const uint4* vb = v != nullptr ? v + row0 * TPR + j : nullptr;
 
   double acc[G][16];
+  uint32_t vm[8];  // two fp16 magnitudes each: channels 8j+2e, +1 (e < 4), then the upper half
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int e = 0; e < 16; ++e) acc[h][e] = 0.0;
-#pragma unroll 1
-  for (int r = r0 + rl; r < r1; r += RPI) {
-    const float* ct = cosT + static_cast<size_t>(r) * H2 + 8 * j;
-    const float* st = sinT + static_cast<size_t>(r) * H2 + 8 * j;
-    const float4 c0 = ld_f4(ct), c1 = ld_f4(ct + 4), s0 = ld_f4(st), s1 = ld_f4(st + 4);
-    uint4 lo[G], hi[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const uint4* row = k + (row0[h] + r) * TPR;
-      lo[h] = ld_stream(row + j);
-      hi[h] = ld_stream(row + j + TP);
+  for (int e = 0; e < 8; ++e) vm[e] = 0;
+#pragma unroll 1
+  for (int r = r0 + rl; r < r1; r += U * RPI) {
+    float4 tc[U][2], ts[U][2];
+    uint4 lo[U][G], hi[U][G], vlo[U], vhi[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int rr = r + u * RPI;
+      const bool in = rr < r1;
+      const float* ct = cosT + static_cast<size_t>(in ? rr : r) * H2 + 8 * j;
+      const float* st = sinT + static_cast<size_t>(in ? rr : r) * H2 + 8 * j;
+      tc[u][0] = ld_f4(ct);
+      tc[u][1] = ld_f4(ct + 4);
+      ts[u][0] = ld_f4(st);
+      ts[u][1] = ld_f4(st + 4);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const uint4* row = kb + h * hstride + static_cast<size_t>(rr) * TPR;
+        lo[u][h] = in ? ld_stream(row) : make_uint4(0, 0, 0, 0);  // rows past the chunk add +0
+        hi[u][h] = in ? ld_stream(row + TP) : make_uint4(0, 0, 0, 0);
+      }
+      if (vb != nullptr) {
+        vlo[u] = in ? ld_stream(vb + static_cast<size_t>(rr) * TPR) : make_uint4(0, 0, 0, 0);
+        vhi[u] = in ? ld_stream(vb + static_cast<size_t>(rr) * TPR + TP) : make_uint4(0, 0, 0, 0);
+      }
     }
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      rope2(lo[h].x, hi[h].x, f2_pack(c0.x, c0.y), f2_pack(s0.x, s0.y));
-      rope2(lo[h].y, hi[h].y, f2_pack(c0.z, c0.w), f2_pack(s0.z, s0.w));
-      rope2(lo[h].z, hi[h].z, f2_pack(c1.x, c1.y), f2_pack(s1.x, s1.y));
-      rope2(lo[h].w, hi[h].w, f2_pack(c1.z, c1.w), f2_pack(s1.z, s1.w));
-      const uint32_t wl[4] = {lo[h].x, lo[h].y, lo[h].z, lo[h].w}, wh[4] = {hi[h].x, hi[h].y, hi[h].z, hi[h].w};
+    for (int u = 0; u < U; ++u) {
+      const float4 c0 = tc[u][0], c1 = tc[u][1], s0 = ts[u][0], s1 = ts[u][1];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        add_f16x2(acc[h][2 * e], acc[h][2 * e + 1], wl[e]);
-        add_f16x2(acc[h][8 + 2 * e], acc[h][8 + 2 * e + 1], wh[e]);
+      for (int h = 0; h < G; ++h) {
+        uint4& l = lo[u][h];
+        uint4& hh = hi[u][h];
+        rope2(l.x, hh.x, f2_pack(c0.x, c0.y), f2_pack(s0.x, s0.y));
+        rope2(l.y, hh.y, f2_pack(c0.z, c0.w), f2_pack(s0.z, s0.w));
+        rope2(l.z, hh.z, f2_pack(c1.x, c1.y), f2_pack(s1.x, s1.y));
+        rope2(l.w, hh.w, f2_pack(c1.z, c1.w), f2_pack(s1.z, s1.w));
+        const uint32_t wl[4] = {l.x, l.y, l.z, l.w}, wh[4] = {hh.x, hh.y, hh.z, hh.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          add_f16x2(acc[h][2 * e], acc[h][2 * e + 1], wl[e]);
+          add_f16x2(acc[h][8 + 2 * e], acc[h][8 + 2 * e + 1], wh[e]);
+        }
+      }
+      if (vb != nullptr) {
+        const uint32_t wl[4] = {vlo[u].x, vlo[u].y, vlo[u].z, vlo[u].w};
+        const uint32_t wh[4] = {vhi[u].x, vhi[u].y, vhi[u].z, vhi[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {  // |fp16| ordered as integers, two per word
+          vm[e] = __vmaxu2(vm[e], wl[e] & 0x7FFF7FFFu);
+          vm[4 + e] = __vmaxu2(vm[4 + e], wh[e] & 0x7FFF7FFFu);
+        }
       }
     }
   }
   // lanes of a warp with the same j hold the same channels: fold them, then
   // the warps through shared memory
 #pragma unroll
-  for (int o = TP; o < 32; o <<= 1)
+  for (int o = TP; o < 32; o <<= 1) {
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
       for (int e = 0; e < 16; ++e) acc[h][e] = __dadd_rn(acc[h][e], __shfl_xor_sync(0xFFFFFFFFu, acc[h][e], o));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) vm[e] = __vmaxu2(vm[e], __shfl_xor_sync(0xFFFFFFFFu, vm[e], o));
+  }
   __shared__ double s_sum[kThreads / 32][G][D];
+  __shared__ uint32_t s_vm[kThreads / 32][D / 2];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane < TP) {
 #pragma unroll
@@ -290,6 +333,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_colstats_rope(const uint4* __re
         s_sum[w][h][8 * j + e] = acc[h][e];
         s_sum[w][h][H2 + 8 * j + e] = acc[h][8 + e];
       }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      s_vm[w][4 * j + e] = vm[e];
+      s_vm[w][H2 / 2 + 4 * j + e] = vm[4 + e];
+    }
   }
   __syncthreads();
   for (int t = threadIdx.x; t < G * D; t += kThreads) {
@@ -298,6 +346,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_colstats_rope(const uint4* __re
 #pragma unroll
     for (int i = 0; i < kThreads / 32; ++i) sum = __dadd_rn(sum, s_sum[i][h][c]);
     ksum[(static_cast<size_t>(z0 + h) * nchunk + chunk) * D + c] = __double2ll_rn(__dmul_rn(sum, 0x1p24));
+  }
+  if (vb != nullptr && threadIdx.x < D) {
+    const int c = threadIdx.x;
+    uint32_t mx = 0;
+#pragma unroll
+    for (int i = 0; i < kThreads / 32; ++i) mx = max(mx, (s_vm[i][c >> 1] >> ((c & 1) * 16)) & 0xFFFFu);
+    vmax[(static_cast<size_t>(z0) * nchunk + chunk) * D + c] = mx;
   }
 }
 
@@ -343,16 +398,6 @@ __global__ void __launch_bounds__(256) k_finalize(const long long* __restrict__ 
   }
 }
 
-// Round-half-even of y to an int8 code: adding 1.5*2^23 leaves the rounded
-// integer in the low mantissa bits (the fp32 add rounds to nearest even at
-// unit spacing), whose low byte is the two's-complement code.  No clamp is
-// needed: |x| <= absmax and delta = RN(absmax / 127) >= absmax/127 * (1 -
-// 2^-24), so |RN(x / delta)| <= 127 * (1 + 2^-22) and rounds to at most 127;
-// -0 and +0 both give code 0.
-__device__ __forceinline__ uint32_t rne_code8(float y) {
-  return __float_as_uint(__fadd_rn(y, 12582912.f)) & 0xFFu;
-}
-
 struct QuantJobs {
   const uint4* q;       // fp16 [B,H,N,D]
   const uint4* k;       // fp16 [B,Hkv,N,D]
@@ -373,10 +418,62 @@ struct QuantJobs {
   int n_q, n_k, n_v;    // number of (slab, block) jobs of each kind
 };
 
+// E4M3 codes of one 128-token block of V (slab, blk): per-channel scale,
+// no block reduction: e4m3(RN(v / delta_v[c])) (div_rn_by of quant_div.h,
+// lane-wise), 0 for a channel whose delta_v is 0.
+template <int D>
+__device__ __forceinline__ void quant_v_block(const QuantJobs& J, int slab, int blk) {
+  constexpr int TPR = D / 8;               // uint4 per token row
+  constexpr int U = 128 * TPR / kThreads;  // uint4 per thread
+  size_t srow;
+  int len;
+  slab_rows(J.seq, slab, J.Hkv, &srow, &len);
+  const int rows = min(128, len - blk * 128);
+  if (rows <= 0) return;  // a block past the end of a short sequence
+  const size_t row0 = srow + static_cast<size_t>(blk) * 128;
+  const uint4* src = J.v + row0 * TPR;
+  uint2* dst = J.v_hat + row0 * TPR;
+  const int cg = threadIdx.x % TPR;  // this thread's 8 channels: cg*8 .. cg*8+7 (fixed across u)
+  uint4 raw[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int idx = threadIdx.x + kThreads * u;
+    raw[u] = (idx / TPR < rows) ? ld_stream(src + idx) : make_uint4(0, 0, 0, 0);
+  }
+  uint64_t nd2[4], r2[4];
+  uint32_t keep[4];  // per channel pair: byte masks of the channels with delta_v != 0
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float d0 = J.delta_v[static_cast<size_t>(slab) * D + cg * 8 + 2 * e];
+    const float d1 = J.delta_v[static_cast<size_t>(slab) * D + cg * 8 + 2 * e + 1];
+    nd2[e] = f2_pack(-d0, -d1);
+    r2[e] = f2_pack(d0 != 0.f ? __frcp_rn(d0) : 0.f, d1 != 0.f ? __frcp_rn(d1) : 0.f);
+    keep[e] = (d0 != 0.f ? 0x00FFu : 0u) | (d1 != 0.f ? 0xFF00u : 0u);  // bytes of the e4m3 pair
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int idx = threadIdx.x + kThreads * u;
+    const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+    uint32_t out[2] = {0, 0};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint64_t x = f2_from_h2(w[e]);
+      const uint64_t q = f2_mul(x, r2[e]);
+      const float2 y = f2_unpack(f2_fma(f2_fma(q, nd2[e], x), r2[e], q));
+      const float2 xf = f2_unpack(x);
+      // the correction's adds turn a -0 quotient into +0: the sign of x is
+      // put back (E4M3 encodes -0 as 0x80)
+      out[e >> 1] |= (pack_e4m3x2(copysignf(y.x, xf.x), copysignf(y.y, xf.y)) & keep[e]) << ((e & 1) * 16);
+    }
+    if (idx / TPR < rows) dst[idx] = make_uint2(out[0], out[1]);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 4) k_quant(const QuantJobs J) {
   constexpr int TPR = D / 8;                  // uint4 per token row
   constexpr int U = 128 * TPR / kThreads;     // uint4 per thread
+  constexpr int RPU = kThreads / TPR;         // rows between a thread's uint4s
   __shared__ float s_red[kThreads / 32];
 
   int job = blockIdx.x;
@@ -387,8 +484,8 @@ __global__ void __launch_bounds__(kThreads, 4) k_quant(const QuantJobs J) {
     kind = 1;
     job -= J.n_q;
   } else {
-    kind = 2;
-    job -= J.n_q + J.n_k;
+    quant_v_block<D>(J, (job - J.n_q - J.n_k) / J.nb, (job - J.n_q - J.n_k) % J.nb);
+    return;
   }
   const int slab = job / J.nb, blk = job % J.nb;
   size_t srow;
@@ -397,9 +494,10 @@ __global__ void __launch_bounds__(kThreads, 4) k_quant(const QuantJobs J) {
   const int rows = min(128, len - blk * 128);
   if (rows <= 0) return;  // a block past the end of a short sequence
   const size_t row0 = srow + static_cast<size_t>(blk) * 128;
-  const uint4* src = (kind == 0 ? J.q : kind == 1 ? J.k : J.v) + row0 * TPR;
-  uint2* dst = (kind == 0 ? J.q_hat : kind == 1 ? J.k_hat : J.v_hat) + row0 * TPR;
+  const uint4* src = (kind == 0 ? J.q : J.k) + row0 * TPR;
+  uint2* dst = (kind == 0 ? J.q_hat : J.k_hat) + row0 * TPR;
   const int cg = threadIdx.x % TPR;  // this thread's 8 channels: cg*8 .. cg*8+7 (fixed across u)
+  const int rl = threadIdx.x / TPR;  // this thread's first row
 
   uint4 raw[U];
 #pragma unroll
@@ -408,58 +506,52 @@ __global__ void __launch_bounds__(kThreads, 4) k_quant(const QuantJobs J) {
     raw[u] = (idx / TPR < rows) ? ld_stream(src + idx) : make_uint4(0, 0, 0, 0);
   }
 
-  if (kind == 2) {
-    // V: per-channel scale, no block reduction.
-    float dv[8], rv[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      dv[e] = J.delta_v[static_cast<size_t>(slab) * D + cg * 8 + e];
-      rv[e] = dv[e] != 0.f ? __frcp_rn(dv[e]) : 0.f;
-    }
+  // x = fp32(q) * sm_scale or fp32(k) - mean_k.  The block absmax is taken
+  // on the fp16 values (rounding is monotonic: max |fl(f s)| = fl(max |f| s)
+  // and, per channel, max |fl(f - m)| = max(|fl(max f - m)|, |fl(min f - m)|)).
+  float amax = 0.f;
+  uint64_t m2[4];
+  if (kind == 0) {
+    uint32_t mag = 0;  // two fp16 magnitudes (rows past the end are +0)
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int idx = threadIdx.x + kThreads * u;
       const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-      uint32_t out[2] = {0, 0};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const __half2 h = *reinterpret_cast<const __half2*>(&w[e]);
-        const float2 f = __half22float2(h);
-        const float y0 = dv[2 * e] != 0.f ? div_rn_by(f.x, dv[2 * e], rv[2 * e]) : 0.f;
-        const float y1 = dv[2 * e + 1] != 0.f ? div_rn_by(f.y, dv[2 * e + 1], rv[2 * e + 1]) : 0.f;
-        out[e >> 1] |= pack_e4m3x2(y0, y1) << ((e & 1) * 16);
-      }
-      if (idx / TPR < rows) dst[idx] = make_uint2(out[0], out[1]);
+      for (int e = 0; e < 4; ++e) mag = __vmaxu2(mag, w[e] & 0x7FFF7FFFu);
     }
-    return;
-  }
-
-  float sub[8];
+    const uint32_t mx = max(mag & 0xFFFFu, mag >> 16);
+    amax = __fmul_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(mx))), fabsf(J.sm_scale));
+  } else {
+    const float* mk = J.mean_k + static_cast<size_t>(slab) * D + cg * 8;
 #pragma unroll
-  for (int e = 0; e < 8; ++e)
-    sub[e] = (kind == 1) ? J.mean_k[static_cast<size_t>(slab) * D + cg * 8 + e] : 0.f;
-
-  // x = fp32(q) * sm_scale or fp32(k) - mean_k, formed twice (for the block
-  // max and for the codes) so that only the raw loads stay live in between
-  auto xval = [&](uint32_t w, int e) -> float2 {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
-    return kind == 0 ? make_float2(__fmul_rn(f.x, J.sm_scale), __fmul_rn(f.y, J.sm_scale))
-                     : make_float2(__fsub_rn(f.x, sub[2 * e]), __fsub_rn(f.y, sub[2 * e + 1]));
-  };
-  float amax = 0.f;
+    for (int e = 0; e < 4; ++e) m2[e] = f2_pack(mk[2 * e], mk[2 * e + 1]);
+    if (rl < rows) {  // u = 0 is this thread's first row; later ones may be past the end
+      __half2 cmax[4], cmin[4];
+      {
+        const uint32_t w[4] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w};
 #pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-    const int idx = threadIdx.x + kThreads * u;
-    if (idx / TPR < rows) {
+        for (int e = 0; e < 4; ++e) cmax[e] = cmin[e] = *reinterpret_cast<const __half2*>(&w[e]);
+      }
+#pragma unroll
+      for (int u = 1; u < U; ++u) {
+        if (rl + u * RPU < rows) {
+          const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __half2 v = *reinterpret_cast<const __half2*>(&w[e]);
+            cmax[e] = __hmax2(cmax[e], v);
+            cmin[e] = __hmin2(cmin[e], v);
+          }
+        }
+      }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 x = xval(w[e], e);
-        amax = fmaxf(amax, fmaxf(fabsf(x.x), fabsf(x.y)));
+        const float2 a = f2_unpack(f2_sub(f2_from_h2(*reinterpret_cast<const uint32_t*>(&cmax[e])), m2[e]));
+        const float2 b = f2_unpack(f2_sub(f2_from_h2(*reinterpret_cast<const uint32_t*>(&cmin[e])), m2[e]));
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(b.x), fabsf(b.y))));
       }
     }
   }
-  // block absmax
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
   if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = amax;
@@ -471,28 +563,25 @@ __global__ void __launch_bounds__(kThreads, 4) k_quant(const QuantJobs J) {
   const float delta = __fdiv_rn(amax, 127.f);
   if (threadIdx.x == 0) (kind == 0 ? J.delta_q : J.delta_k)[static_cast<size_t>(slab) * J.nb + blk] = delta;
   const float r = delta != 0.f ? __frcp_rn(delta) : 0.f;
-
+  const uint64_t r2 = f2_pack(r, r), nd2 = f2_pack(-delta, -delta), s2 = f2_pack(J.sm_scale, J.sm_scale);
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     const int idx = threadIdx.x + kThreads * u;
+    if (idx / TPR >= rows) continue;
     const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-    uint32_t out[2];
+    uint64_t x[4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const float2 x0 = xval(w[2 * h], 2 * h), x1 = xval(w[2 * h + 1], 2 * h + 1);
-      const float xs[4] = {x0.x, x0.y, x1.x, x1.y};
-      uint32_t b[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) b[e] = delta != 0.f ? rne_code8(div_rn_nosign(xs[e], delta, r)) : 0u;
-      out[h] = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-    }
-    if (idx / TPR < rows) dst[idx] = make_uint2(out[0], out[1]);
+    for (int e = 0; e < 4; ++e) x[e] = kind == 0 ? f2_mul(f2_from_h2(w[e]), s2) : f2_sub(f2_from_h2(w[e]), m2[e]);
+    uint2 out = make_uint2(0u, 0u);
+    if (delta != 0.f) out = make_uint2(codes4(x[0], x[1], nd2, r2), codes4(x[2], x[3], nd2, r2));
+    dst[idx] = out;
   }
 }
 
 // Q and K blocks with rotary embedding: one CTA per (128-token block, G
 // consecutive heads of one batch entry, Q or K); jobs [0, n_q) are Q
-// groups, [n_q, n_q + n_k) K groups.  The block's cos / sin rows are staged
+// groups, [n_q, n_q + n_k) K groups, then n_v V blocks (one head each, no
+// rotation, as in k_quant).  The block's cos / sin rows are staged
 // once in shared memory, then each head's block is rotated and quantized
 // with the values of k_quant: x = fp32(q) * sm_scale or fp32(k) - mean_k,
 // delta = RN(absmax / 127), codes RN(x / delta).  A thread holds channel
@@ -514,6 +603,11 @@ __global__ void __launch_bounds__(kThreads, 3) k_quant_rope(const QuantJobs J) {
   __shared__ float s_red[2][kThreads / 32];
 
   int job = blockIdx.x;
+  if (job >= J.n_q + J.n_k) {  // V: no rotation
+    job -= J.n_q + J.n_k;
+    quant_v_block<D>(J, job / J.nb, job % J.nb);
+    return;
+  }
   const int kind = job < J.n_q ? 0 : 1;
   if (kind == 1) job -= J.n_q;
   const int Hs = kind == 0 ? J.H : J.Hkv;
@@ -679,17 +773,25 @@ cudaError_t launch_colstats(const void* k, const void* v, int slabs, int N, int 
   const uint4* k4 = static_cast<const uint4*>(k);
   const uint4* v4 = static_cast<const uint4*>(v);
   if (cos_t != nullptr && k != nullptr) {
-    // rotated K sums per head group; V maxima (if any) by the plain kernel
-    const int G = Hkv % 2 == 0 ? 2 : 1;
-    const dim3 grid(nchunk, slabs / G);
-    if (D == 128) {
-      if (G == 2) k_colstats_rope<128, 2><<<grid, kThreads, 0, st>>>(k4, seq, Hkv, nchunk, ksum, cos_t, sin_t);
-      else k_colstats_rope<128, 1><<<grid, kThreads, 0, st>>>(k4, seq, Hkv, nchunk, ksum, cos_t, sin_t);
+    // rotated K sums, with the V maxima in the same pass; without V, K of
+    // two heads per CTA share the table loads
+    if (v4 != nullptr) {
+      const dim3 grid(nchunk, slabs);
+      if (D == 128) k_colstats_rope<128, 1, 2><<<grid, kThreads, 0, st>>>(k4, v4, seq, Hkv, nchunk, ksum, vmax, cos_t, sin_t);
+      else k_colstats_rope<64, 1, 2><<<grid, kThreads, 0, st>>>(k4, v4, seq, Hkv, nchunk, ksum, vmax, cos_t, sin_t);
     } else {
-      if (G == 2) k_colstats_rope<64, 2><<<grid, kThreads, 0, st>>>(k4, seq, Hkv, nchunk, ksum, cos_t, sin_t);
-      else k_colstats_rope<64, 1><<<grid, kThreads, 0, st>>>(k4, seq, Hkv, nchunk, ksum, cos_t, sin_t);
+      const int G = Hkv % 2 == 0 ? 2 : 1;
+      const dim3 grid(nchunk, slabs / G);
+      if (D == 128) {
+        if (G == 2) k_colstats_rope<128, 2, 1><<<grid, kThreads, 0, st>>>(k4, nullptr, seq, Hkv, nchunk, ksum, nullptr, cos_t, sin_t);
+        else k_colstats_rope<128, 1, 2><<<grid, kThreads, 0, st>>>(k4, nullptr, seq, Hkv, nchunk, ksum, nullptr, cos_t, sin_t);
+      } else {
+        if (G == 2) k_colstats_rope<64, 2, 1><<<grid, kThreads, 0, st>>>(k4, nullptr, seq, Hkv, nchunk, ksum, nullptr, cos_t, sin_t);
+        else k_colstats_rope<64, 1, 2><<<grid, kThreads, 0, st>>>(k4, nullptr, seq, Hkv, nchunk, ksum, nullptr, cos_t, sin_t);
+      }
     }
     k4 = nullptr;
+    v4 = nullptr;
     ksum = nullptr;
   }
   if (k4 != nullptr || v4 != nullptr) {
@@ -765,13 +867,12 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st) {
   J.n_v = a.v ? a.B * a.H_kv * J.nb : 0;
   if (J.n_q + J.n_k + J.n_v == 0) return cudaSuccess;
   if (a.cos_t != nullptr && J.n_q + J.n_k > 0) {
-    // Q and K in head groups with the rotary table; V below on its own
+    // Q and K in head groups with the rotary table, V blocks after them
     const int G = std::min(rope_group(a.H), rope_group(a.H_kv));
     QuantJobs R = J;
     R.n_q = J.n_q / G;
     R.n_k = J.n_k / G;
-    R.n_v = 0;
-    const int total = R.n_q + R.n_k;
+    const int total = R.n_q + R.n_k + R.n_v;
     cudaError_t e;
     if (a.d == 128) {
       e = G == 4 ? launch_quant_rope<128, 4>(R, total, st)
@@ -783,6 +884,7 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     J.n_q = 0;
     J.n_k = 0;
+    J.n_v = 0;
   }
   const int total = J.n_q + J.n_k + J.n_v;
   if (total > 0) {
