@@ -60,6 +60,8 @@ NCU_TRAFFIC = {
     # 638.5 MB on the same small case: persistent scheduler, one CTA per item
     # for long non-causal shapes
     ("961ce71c0f592454", "video_dit_h24_n32768_d128", "8+8"): 478.9e6,
+    # 638.5 MB on the same small case (8+8 scores converted with cvt)
+    ("9c9600bbb5e83058", "video_dit_h24_n32768_d128", "8+8"): 478.9e6,
 }
 
 

@@ -356,24 +356,27 @@ __global__ void __launch_bounds__(kThreads, 2) k_colstats_rope(const uint4* __re
   }
 }
 
-// One CTA per (slab, 32 channels): its 8 warps reduce interleaved chunks
-// (lane = channel), then warp 0 combines them.  Integer sums and maxima are
-// exact, so the result does not depend on this order.
-__global__ void __launch_bounds__(256) k_finalize(const long long* __restrict__ ksum,
-                                                  const uint32_t* __restrict__ vmax, int nchunk_max,
-                                                  int D, SeqLayout seq, int Hkv, float v_r,
-                                                  float* __restrict__ mean_k, float* __restrict__ delta_v) {
+// One CTA per (slab, 32 channels): its kFinWarps warps reduce interleaved
+// chunks (lane = channel, several loads in flight per lane), then warp 0
+// combines them.  Integer sums and maxima are exact, so the result does not
+// depend on this order.
+constexpr int kFinWarps = 16;
+__global__ void __launch_bounds__(kFinWarps * 32) k_finalize(const long long* __restrict__ ksum,
+                                                             const uint32_t* __restrict__ vmax, int nchunk_max,
+                                                             int D, SeqLayout seq, int Hkv, float v_r,
+                                                             float* __restrict__ mean_k, float* __restrict__ delta_v) {
   const int slab = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int c = blockIdx.y * 32 + lane;
   size_t row0;
   int N;
   slab_rows(seq, slab, Hkv, &row0, &N);
   const int nchunk = (N + kStatRows - 1) / kStatRows;  // chunks written for this slab
-  __shared__ long long s_s[8][32];
-  __shared__ uint32_t s_m[8][32];
+  __shared__ long long s_s[kFinWarps][32];
+  __shared__ uint32_t s_m[kFinWarps][32];
   long long s = 0;
   uint32_t m = 0;
-  for (int i = w; i < nchunk; i += 8) {
+#pragma unroll 4
+  for (int i = w; i < nchunk; i += kFinWarps) {
     const size_t o = (static_cast<size_t>(slab) * nchunk_max + i) * D + c;
     if (ksum != nullptr) s += ksum[o];
     if (vmax != nullptr) m = max(m, vmax[o]);
@@ -383,7 +386,7 @@ __global__ void __launch_bounds__(256) k_finalize(const long long* __restrict__ 
   __syncthreads();
   if (w != 0) return;
 #pragma unroll
-  for (int i = 1; i < 8; ++i) {
+  for (int i = 1; i < kFinWarps; ++i) {
     s += s_s[i][lane];
     m = max(m, s_m[i][lane]);
   }
@@ -810,7 +813,7 @@ cudaError_t launch_finalize(const long long* ksum, const uint32_t* vmax, int sla
   seq = fixed_or(seq, N);
   const int nchunk = static_cast<int>(stat_chunks(seq.max_len));
   if (slabs == 0) return cudaSuccess;
-  k_finalize<<<dim3(slabs, D / 32), 256, 0, st>>>(ksum, vmax, nchunk, D, seq, Hkv, v_r, mean_k, delta_v);
+  k_finalize<<<dim3(slabs, D / 32), kFinWarps * 32, 0, st>>>(ksum, vmax, nchunk, D, seq, Hkv, v_r, mean_k, delta_v);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) set_error_detail("finalize kernel launch", e);
   return e;
