@@ -62,6 +62,8 @@ NCU_TRAFFIC = {
     ("961ce71c0f592454", "video_dit_h24_n32768_d128", "8+8"): 478.9e6,
     # 638.5 MB on the same small case (8+8 scores converted with cvt)
     ("9c9600bbb5e83058", "video_dit_h24_n32768_d128", "8+8"): 478.9e6,
+    # 641.8 MB on the same small case (conversion chosen per shape at launch)
+    ("856f3b58769ce495", "video_dit_h24_n32768_d128", "8+8"): 481.3e6,
 }
 
 

@@ -241,7 +241,7 @@ __device__ __forceinline__ int tile_rowmax(uint32_t (&a)[128], int lim) {
 // holds the s32 scores on entry and the packed P operand on exit (fp16x2, or
 // 4 x e4m3 per word; lower columns in lower bits).  Returns the row sum of
 // the unrounded P values.
-template <int VAR, bool MASKED>
+template <int VAR, bool MASKED, bool CVT>
 __device__ __forceinline__ float tile_exp(uint32_t (&a)[128], float c, float bias, int lim) {
   const uint64_t c2 = pk2(c, c), b2 = pk2(bias, bias), magic2 = pk2(-kMagic, -kMagic);
   uint64_t sum2[4];
@@ -252,12 +252,12 @@ __device__ __forceinline__ float tile_exp(uint32_t (&a)[128], float c, float bia
     float p[4];
 #pragma unroll
     for (int e = 0; e < 4; e += 2) {
-      // acc as fp32, exactly (|acc| < 2^22).  8+8: a plain conversion;
-      // variant B: kMagicBits + acc reads as the fp32 value 1.5 * 2^23 + acc
-      // and one subtraction gives acc (each form measured faster in its
-      // variant's loop)
+      // acc as fp32, exactly (|acc| < 2^22): CVT, a plain conversion (ALU
+      // pipe), else kMagicBits + acc, which reads as the fp32 value
+      // 1.5 * 2^23 + acc, and one subtraction (FMA pipe); the kernel picks
+      // the form measured faster for its variant and shape
       uint64_t f2;
-      if (VAR == 1) {
+      if (CVT) {
         f2 = pk2(static_cast<float>(static_cast<int>(a[i + e])), static_cast<float>(static_cast<int>(a[i + e + 1])));
       } else {
         f2 = add2(pk2(__uint_as_float(a[i + e] + kMagicBits), __uint_as_float(a[i + e + 1] + kMagicBits)), magic2);
@@ -282,7 +282,7 @@ __device__ __forceinline__ float tile_exp(uint32_t (&a)[128], float c, float bia
   return s.x + s.y;
 }
 
-template <int D, int VAR, bool CAUSAL, bool PACKED>
+template <int D, int VAR, bool CAUSAL, bool PACKED, bool CVT>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, const AttnKParams p) {
@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         s_alpha[(g * PB + u % PB) * 128 + r] = alpha;
         mbar_arrive(&a_full[g * PB + u % PB]);
         const float bias = (VAR == 1) ? (p.log2_pr - m_new) : -m_new;
-        const float rs = masked ? tile_exp<VAR, true>(a, c, bias, lim) : tile_exp<VAR, false>(a, c, bias, lim);
+        const float rs = masked ? tile_exp<VAR, true, CVT>(a, c, bias, lim) : tile_exp<VAR, false, CVT>(a, c, bias, lim);
         l = __fmaf_rn(alpha, l, rs);
         if (C::PS) {
           // row r, 16-byte chunk k (keys 16k..16k+15) at the 128-byte-swizzled
@@ -858,12 +858,12 @@ static cudaError_t sm_count(int* out) {
   return cudaSuccess;
 }
 
-template <int D, int VAR, bool CAUSAL, bool PACKED>
+template <int D, int VAR, bool CAUSAL, bool PACKED, bool CVT>
 static cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   using C = Cfg<D, VAR>;
   // the dynamic shared-memory limit is a per-device function attribute
   static std::atomic<bool> attr_set[kMaxDevices];
-  auto kern = k_attn<D, VAR, CAUSAL, PACKED>;
+  auto kern = k_attn<D, VAR, CAUSAL, PACKED, CVT>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -926,15 +926,22 @@ static cudaError_t launch_t(const AttnArgs& a, cudaStream_t st) {
   return e;
 }
 
+// Score conversion (tile_exp's CVT) by measurement: the plain conversion
+// for 8+8 at d = 128 and for 8+8 at d = 64 up to 8192 keys; the magic-number
+// form for variant B and for longer d = 64 sequences.
 template <bool PACKED>
 static cudaError_t launch_p(const AttnArgs& a, cudaStream_t st) {
   const bool c = a.causal != 0;
   if (a.d == 128) {
-    if (a.variant == 0) return c ? launch_t<128, 0, true, PACKED>(a, st) : launch_t<128, 0, false, PACKED>(a, st);
-    return c ? launch_t<128, 1, true, PACKED>(a, st) : launch_t<128, 1, false, PACKED>(a, st);
+    if (a.variant == 0)
+      return c ? launch_t<128, 0, true, PACKED, false>(a, st) : launch_t<128, 0, false, PACKED, false>(a, st);
+    return c ? launch_t<128, 1, true, PACKED, true>(a, st) : launch_t<128, 1, false, PACKED, true>(a, st);
   }
-  if (a.variant == 0) return c ? launch_t<64, 0, true, PACKED>(a, st) : launch_t<64, 0, false, PACKED>(a, st);
-  return c ? launch_t<64, 1, true, PACKED>(a, st) : launch_t<64, 1, false, PACKED>(a, st);
+  if (a.variant == 0)
+    return c ? launch_t<64, 0, true, PACKED, false>(a, st) : launch_t<64, 0, false, PACKED, false>(a, st);
+  if (a.N <= 8192)
+    return c ? launch_t<64, 1, true, PACKED, true>(a, st) : launch_t<64, 1, false, PACKED, true>(a, st);
+  return c ? launch_t<64, 1, true, PACKED, false>(a, st) : launch_t<64, 1, false, PACKED, false>(a, st);
 }
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
