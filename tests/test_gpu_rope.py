@@ -100,3 +100,31 @@ def test_rope_attention_matches_mirror(sage):
         c_gpu, c_mirror = oracle.cossim(o.cpu().numpy(), ref), oracle.cossim(mirror, ref)
         assert c_gpu >= c_mirror - 1e-4, (variant, c_gpu, c_mirror)
         assert c_mirror >= 0.99, (variant, c_mirror)
+
+
+def test_rope_attention_bias_after_rotation(sage):
+    """The channel-wise K bias that Smooth K removes is the one the pages
+    observe in the K that enters attention, i.e. after the rotation.  Inputs
+    here are the recipe's q, k rotated backwards (cos, -sin), so that the
+    fused rotation hands the quantizers the recipe's biased K: the rotated
+    pre-pass plus attention must then meet the full accuracy bar (CosSim >=
+    0.998 against fp64 attention of the rotated inputs) as well as criterion
+    (b) against the quantized mirror."""
+    w = workloads.get("small_b_n256_d64").with_(N=384, H=4, H_kv=2, seed=77)
+    q, k, v = workloads.generate(w)
+    cos, sin = workloads.rope_tables(w.N, w.d)
+    qpre, kpre = oracle.rope(q, cos, -sin), oracle.rope(k, cos, -sin)
+    for variant in ("B", "8+8"):
+        got, (qr, kr) = check_rope_prepass(sage, qpre, kpre, v, w.scale)
+        qh, kh, dq, dk, _, vh, dv = got
+        tv, = to_dev(v)
+        o = sage.sage_attn_fwd_quantized(qh, kh, dq, dk, vh if variant == "8+8" else tv,
+                                         dv if variant == "8+8" else None, causal=False,
+                                         variant=variant)
+        torch.cuda.synchronize()
+        mirror, inter = oracle.sage_attention(qr, kr, v, causal=False, sm_scale=w.scale,
+                                              variant=variant, ambiguity=EPS_P)
+        err = np.abs(o.cpu().numpy().astype(np.float64) - mirror.astype(np.float64))
+        assert np.all(err <= TOL_B + inter["slack"]), (variant, float(err.max()))
+        ref = oracle.attention_reference(qr, kr, v, causal=False, sm_scale=w.scale)
+        assert oracle.cossim(o.cpu().numpy(), ref) >= 0.998, variant
