@@ -220,7 +220,11 @@ sage_status_t sage_attn_fwd_ws(const void* q, const void* k, const void* v, void
  * kernels on `stream`, copies out on a second internal stream, so one
  * chunk's transfers overlap another chunk's kernels.  The results equal
  * sage_attn_fwd's.  Device buffers are stream-ordered allocations on
- * `stream`, freed before return.
+ * `stream`, freed before return.  The two internal streams and their events
+ * are created on a device's first call and reused by later calls (a call
+ * made while another one holds them on the same device creates and
+ * destroys its own); after cudaDeviceReset the library must be reloaded
+ * before the next call on that device.
  */
 sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
                                  void* o_host, int B, int H, int H_kv, int N, int d, int causal,

@@ -13,20 +13,22 @@ namespace {
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
 
 constexpr int kMaxDevices = 64;
-int g_dev_ok[kMaxDevices];  // 0 unknown, 1 sm_100, -1 other
+std::atomic<int> g_dev_ok[kMaxDevices];  // 0 unknown, 1 sm_100, -1 other
 
 sage_status_t check_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return SAGE_ERR_DEVICE;
-  if (g_dev_ok[dev] == 0) {
+  int ok = g_dev_ok[dev].load(std::memory_order_acquire);
+  if (ok == 0) {
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
       return SAGE_ERR_CUDA;
-    g_dev_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    ok = (major == 10 && minor == 0) ? 1 : -1;
+    g_dev_ok[dev].store(ok, std::memory_order_release);  // every thread computes the same value
   }
-  return g_dev_ok[dev] == 1 ? SAGE_OK : SAGE_ERR_DEVICE;
+  return ok == 1 ? SAGE_OK : SAGE_ERR_DEVICE;
 }
 
 bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -489,6 +491,37 @@ sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* o
   return from_cuda(ef);
 }
 
+namespace {
+
+// Side streams and events of sage_attn_fwd_host, created once per device
+// and reused by the call that holds the device's lock; a concurrent call on
+// the same device makes its own and destroys them afterwards.
+constexpr int kHostChunks = 8;
+struct HostPipe {
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev[2 * kHostChunks + 2] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_pipe_mu[kMaxDevices];
+
+cudaError_t pipe_create(HostPipe* P) {
+  cudaError_t e = cudaStreamCreateWithFlags(&P->s_in, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&P->s_out, cudaStreamNonBlocking);
+  for (int i = 0; e == cudaSuccess && i < 2 * kHostChunks + 2; ++i)
+    e = cudaEventCreateWithFlags(&P->ev[i], cudaEventDisableTiming);
+  return e;
+}
+
+void pipe_destroy(HostPipe* P) {
+  for (int i = 0; i < 2 * kHostChunks + 2; ++i)
+    if (P->ev[i]) cudaEventDestroy(P->ev[i]);
+  if (P->s_in) cudaStreamDestroy(P->s_in);
+  if (P->s_out) cudaStreamDestroy(P->s_out);
+  *P = HostPipe();
+}
+
+}  // namespace
+
 sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
                                  void* o_host, int B, int H, int H_kv, int N, int d, int causal,
                                  float sm_scale, int variant, void* stream) {
@@ -508,7 +541,7 @@ sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const v
   // tensor.  Chunks of units are pipelined: copies in on one stream, the
   // pass on `stream`, copies out on a third, so the transfers of one chunk
   // overlap the kernels of another.
-  constexpr int kMaxChunks = 8;
+  constexpr int kMaxChunks = kHostChunks;
   const int units = B * H_kv, r = H / H_kv;
   const int nchunk = units < kMaxChunks ? units : kMaxChunks;
   const int per = (units + nchunk - 1) / nchunk;
@@ -519,12 +552,22 @@ sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const v
   const size_t off_k = align256(qb), off_v = off_k + align256(kb), off_o = off_v + align256(kb);
   const size_t off_ws = off_o + align256(qb);
 
-  cudaStream_t s_in = nullptr, s_out = nullptr;
-  cudaEvent_t ev[2 * kMaxChunks + 2] = {};
-  cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
-  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
-  for (int i = 0; e == cudaSuccess && i < 2 * nchunk + 2; ++i)
-    e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);  // in [0, kMaxDevices): check_device passed
+  if (e != cudaSuccess) return from_cuda(e);
+  std::unique_lock<std::mutex> lock(g_pipe_mu[dev], std::try_to_lock);
+  HostPipe own;
+  HostPipe* P = lock.owns_lock() ? &g_pipe[dev] : &own;
+  if (P->s_in == nullptr) {
+    e = pipe_create(P);
+    if (e != cudaSuccess) {
+      pipe_destroy(P);
+      sage::set_error_detail("sage_attn_fwd_host streams", e);
+      return from_cuda(e);
+    }
+  }
+  cudaStream_t s_in = P->s_in, s_out = P->s_out;
+  cudaEvent_t* ev = P->ev;
   cudaEvent_t* ev_in = ev;               // [nchunk] inputs of chunk c on the device
   cudaEvent_t* ev_done = ev + nchunk;    // [nchunk] output of chunk c computed
   cudaEvent_t ev_alloc = ev[2 * nchunk], ev_out = ev[2 * nchunk + 1];
@@ -573,10 +616,7 @@ sage_status_t sage_attn_fwd_host(const void* q_host, const void* k_host, const v
   cudaError_t ef = allocated ? cudaFreeAsync(buf, st) : cudaSuccess;
   cudaError_t es = cudaStreamSynchronize(st);
   if (s_out) cudaStreamSynchronize(s_out);
-  for (int i = 0; i < 2 * nchunk + 2; ++i)
-    if (ev[i]) cudaEventDestroy(ev[i]);
-  if (s_in) cudaStreamDestroy(s_in);
-  if (s_out) cudaStreamDestroy(s_out);
+  if (P == &own) pipe_destroy(&own);
   if (s != SAGE_OK) return s;
   if (e != cudaSuccess) {
     sage::set_error_detail("sage_attn_fwd_host pipeline", e);

@@ -150,6 +150,39 @@ def test_host_pipeline_equals_device_path(sage, shape):
     assert torch.equal(sage.sage_attn_fwd(tq, tk, tv, causal=causal, variant="8+8").cpu(), ho)
 
 
+def test_host_path_concurrent_calls(sage):
+    """Two host threads call sage_attn_fwd_host at once on the same device:
+    one uses the device's cached side streams, the other its own; both
+    outputs equal the device path's, call after call."""
+    import threading
+    w = workloads.get("llm_8p8_b2_h16_n4096_d128").with_(B=2, H=4, H_kv=2, N=700, seed=61)
+    q, k, v = workloads.generate(w)
+    tq, tk, tv = to_dev(q, k, v)
+    ref = sage.sage_attn_fwd(tq, tk, tv, causal=False, variant="8+8").cpu()
+    hq, hk, hv = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
+    outs = [torch.empty(hq.shape, dtype=torch.float16).pin_memory() for _ in range(2)]
+    errors = []
+
+    def run(i):
+        try:
+            torch.cuda.set_device(0)
+            for _ in range(6):
+                outs[i].zero_()
+                sage.sage_attn_fwd_host(hq, hk, hv, outs[i], causal=False, variant="8+8")
+                if not torch.equal(outs[i], ref):
+                    errors.append(i)
+        except Exception as ex:  # surfaced below
+            errors.append(repr(ex))
+
+    threads = [threading.Thread(target=run, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not any(t.is_alive() for t in threads)
+    assert not errors, errors
+
+
 def test_repeated_calls_are_deterministic(sage):
     w = workloads.get("prefill_gqa_causal_h32_kv8_n8192_d128").with_(H=8, H_kv=2, N=2048)
     q, k, v = workloads.generate(w)
