@@ -1,5 +1,7 @@
-// quant_div.h -- the quantizers' division, shared by the pre-pass kernels and
-// the host program that checks it against IEEE division bit for bit.
+// quant_div.h -- the quantizers' division, scalar form: the definition the
+// pre-pass kernels follow (they run the same three steps on two lanes per
+// fp32-pair instruction, each lane rounded as here) and that the host
+// program checks against IEEE division bit for bit.
 //
 // The quantizers need x / delta rounded to nearest ([SA2++] "核心公式":
 // A_hat = round(A / delta), delta_V = colmax|V| / V_r), one division per
