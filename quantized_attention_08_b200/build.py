@@ -13,7 +13,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libsage.so")
 SOURCES = ["prepass.cu", "attn_sm100.cu", "sage_api.cu"]
-HEADERS = ["sage_ptx.cuh", "sage_internal.h", "quant_div.h"]
+HEADERS = ["sage_ptx.cuh", "sage_internal.h", "quant_div.h", "quant_pair.cuh"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

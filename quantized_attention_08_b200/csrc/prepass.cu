@@ -33,6 +33,7 @@
 #include <atomic>
 #include <type_traits>
 
+#include "quant_pair.cuh"
 #include "sage_internal.h"
 
 namespace sage {
@@ -137,69 +138,6 @@ __global__ void __launch_bounds__(kThreads) k_colstats(const uint4* __restrict__
     if (k != nullptr) ksum[o] = __double2ll_rn(__dmul_rn(s, 0x1p24));  // an integer: exact
     if (v != nullptr) vmax[o] = mx;
   }
-}
-
-// ---------------------------------------------------------------- fp32 pairs
-// Lane-wise IEEE fp32 operations on two values (each lane rounded to nearest
-// even, exactly as the scalar operation), two per instruction.  A product
-// must not feed f2_add / f2_sub directly (see rope2).
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-// the two fp16 values of w as fp32 (exact)
-__device__ __forceinline__ uint64_t f2_from_h2(uint32_t w) {
-  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
-  return f2_pack(f.x, f.y);
-}
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-// int8 codes of four x values (two lanes each), delta > 0, r = RN(1/delta),
-// nd = -delta: y = RN(x / delta) (div_rn_nosign of quant_div.h, lane-wise:
-// the remainder fma(q, -delta, x) is the same exact value as fma(-q, delta,
-// x)), then rounded half-even to an integer: adding 1.5 * 2^23 leaves it in
-// the low mantissa bits, whose low byte is the two's-complement code; bytes
-// in lane order.  No clamp is needed: |x| <= absmax and delta = RN(absmax /
-// 127) >= absmax / 127 * (1 - 2^-24), so |y| <= 127 * (1 + 2^-22) rounds to
-// at most 127; -0 and +0 both give code 0.
-__device__ __forceinline__ uint32_t codes4(uint64_t x01, uint64_t x23, uint64_t nd2, uint64_t r2) {
-  const uint64_t magic2 = f2_pack(12582912.f, 12582912.f);
-  const uint64_t q01 = f2_mul(x01, r2), q23 = f2_mul(x23, r2);
-  const uint64_t y01 = f2_fma(f2_fma(q01, nd2, x01), r2, q01);
-  const uint64_t y23 = f2_fma(f2_fma(q23, nd2, x23), r2, q23);
-  const uint64_t c01 = f2_add(y01, magic2), c23 = f2_add(y23, magic2);
-  const uint32_t lo = prmt(static_cast<uint32_t>(c01), static_cast<uint32_t>(c01 >> 32), 0x0040u);
-  const uint32_t hi = prmt(static_cast<uint32_t>(c23), static_cast<uint32_t>(c23 >> 32), 0x0040u);
-  return prmt(lo, hi, 0x5410u);
 }
 
 // Rotary embedding, rotate-half pairing (channel i < D/2 pairs with
@@ -461,8 +399,7 @@ __device__ __forceinline__ void quant_v_block(const QuantJobs& J, int slab, int 
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const uint64_t x = f2_from_h2(w[e]);
-      const uint64_t q = f2_mul(x, r2[e]);
-      const float2 y = f2_unpack(f2_fma(f2_fma(q, nd2[e], x), r2[e], q));
+      const float2 y = f2_unpack(div2_rn(x, nd2[e], r2[e]));
       const float2 xf = f2_unpack(x);
       // the correction's adds turn a -0 quotient into +0: the sign of x is
       // put back (E4M3 encodes -0 as 0x80)
