@@ -160,27 +160,100 @@ def whole_job_tops(ops_per_rank: float, world: int, ms: float) -> float:
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """SM clock and throttle-reason sampling during the timed region.
+
+    NVML (the library nvidia-smi reads) polled every `period_s` from a
+    thread, so that even a region of a few milliseconds gets samples; if
+    NVML is unavailable, an `nvidia-smi --query-gpu ... -lms 100` process.
+    `nvml` may be given a stand-in module (tests)."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits reported here
+    REASON_BITS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+                   ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, period_s: float = 0.002, nvml=None):
         self.index = index
+        self.period = period_s
+        self.nvml = nvml
         self.proc = None
+        self.thread = None
+        self.rows = []
+        self.source = None
+        self.out = ""
+
+    def _handle(self, nv):
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.index).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _start_nvml(self) -> bool:
+        nv = self.nvml
+        if nv is None:
+            try:
+                import pynvml as nv
+            except ImportError:
+                return False
+        try:
+            nv.nvmlInit()
+        except Exception:
+            return False
+        try:
+            h = self._handle(nv)
+            max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            sample = lambda: (float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), max_mhz,  # noqa: E731
+                              int(reasons(h)))
+            self.rows.append(sample())
+        except Exception:
+            nv.nvmlShutdown()
+            return False
+        import threading
+        self.stop = threading.Event()
+
+        def loop():
+            while not self.stop.wait(self.period):
+                try:
+                    self.rows.append(sample())
+                except Exception:
+                    return
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
+        self.nv, self.source = nv, "nvml"
+        return True
 
     def __enter__(self):
+        if self._start_nvml():
+            return self
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
                  "-i", str(self.index), "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi"
         except OSError:
             self.proc = None
         return self
 
     def __exit__(self, *exc):
-        self.out = ""
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
+            try:
+                self.rows.append((float(self.nv.nvmlDeviceGetClockInfo(self._handle(self.nv), self.nv.NVML_CLOCK_SM)),
+                                  self.rows[0][1], self.rows[-1][2]))
+            except Exception:
+                pass
+            try:
+                self.nv.nvmlShutdown()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -190,8 +263,12 @@ class ClockSampler:
                 self.out, _ = self.proc.communicate()
 
     def summary(self):
+        names = [n for n, _ in self.REASON_BITS]
         rows = []
-        for line in (getattr(self, "out", "") or "").splitlines():
+        if self.source == "nvml":
+            for mhz, mx, bits in self.rows:
+                rows.append((mhz, mx, ["Active" if bits & b else "Not Active" for _, b in self.REASON_BITS]))
+        for line in (self.out or "").splitlines():
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
@@ -201,10 +278,9 @@ class ClockSampler:
                 continue
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i] == "Active"})
         return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": self.source}
 
 
 class OracleSampler:
