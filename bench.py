@@ -589,7 +589,7 @@ def main():
             "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_avg},
             "gpu_launches": 4 * args.steps,
-            "clocks": {k_: clocks[k_] for k_ in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "clocks": {k_: clocks.get(k_) for k_ in ("sm_mhz", "sm_max_mhz", "reasons", "samples", "source")},
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
