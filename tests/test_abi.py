@@ -92,6 +92,44 @@ def test_host_argument_checks_need_no_gpu(lib):
     assert r(*args(fake, fake)[:5], 1, 2, 2, 128, 96, *args(fake, fake)[10:]) == 2
 
 
+def test_varlen_and_host_argument_checks_need_no_gpu(lib):
+    """The packed-batch and host-buffer entry points reject bad arguments
+    before any CUDA call (status codes of include/sage.h: 1 invalid,
+    2 unsupported, 3 misaligned), and an empty batch is a no-op."""
+    fake = ctypes.c_void_p(1 << 20)
+    cu = ctypes.c_void_p(1 << 16)
+    f = lib.sage_attn_fwd_varlen
+    # (q, k, v, o, cu_seqlens, B, max_seqlen, T, H, H_kv, d, causal, sm_scale, variant, stream)
+    ok = [fake, fake, fake, fake, cu, 2, 128, 200, 2, 2, 64, 0, 0.125, 1, None]
+
+    def call(**kw):
+        a = list(ok)
+        for i, key in enumerate(("q", "k", "v", "o", "cu", "B", "max_seqlen", "T", "H", "H_kv", "d",
+                                 "causal", "sm_scale", "variant")):
+            if key in kw:
+                a[i] = kw[key]
+        return f(*a)
+
+    assert call(cu=None) == 1                                  # no offsets for a non-empty batch
+    assert call(cu=ctypes.c_void_p((1 << 16) + 2)) == 3        # offsets not 4-byte aligned
+    assert call(T=-1) == 1
+    assert call(T=(1 << 30) + 1) == 2                          # row coordinates are 32-bit
+    assert call(d=96) == 2
+    assert call(variant=7) == 2
+    assert call(causal=2) == 1
+    assert call(sm_scale=0.0) == 1
+    assert call(q=None) == 1
+    assert call(o=ctypes.c_void_p((1 << 20) + 8)) == 3
+    assert call(B=0, cu=None) == 0                             # empty batch
+    assert call(T=0, cu=None) == 0
+    h = lib.sage_attn_fwd_host
+    # (q, k, v, o, B, H, H_kv, N, d, causal, sm_scale, variant, stream)
+    assert h(None, fake, fake, fake, 1, 2, 2, 128, 64, 0, 0.125, 1, None) == 1
+    assert h(fake, fake, fake, fake, 1, 2, 2, 128, 96, 0, 0.125, 1, None) == 2
+    assert h(fake, fake, fake, fake, 1, 2, 2, 128, 64, 0, -1.0, 1, None) == 1
+    assert h(None, None, None, None, 0, 2, 2, 128, 64, 0, 0.125, 1, None) == 0
+
+
 def test_size_limits_are_rejected_before_any_cuda_call(lib):
     """The documented limits: B*H <= 65535 (grid.y) and N <= 2^24 (32-bit
     TMA coordinates); one past each is SAGE_ERR_UNSUPPORTED.  (Only calls
