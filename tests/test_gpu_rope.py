@@ -69,6 +69,34 @@ def test_rope_prepass_bit_exact_small(sage, shape):
     check_rope_prepass(sage, q, k, v, 1.0 / np.sqrt(d))
 
 
+@pytest.mark.parametrize("shape", [(1, 4, 2, 300, 128), (2, 6, 3, 130, 64), (1, 8, 4, 256, 64)],
+                         ids=lambda s: "B{}_H{}_Hkv{}_N{}_d{}".format(*s))
+def test_rope_prepass_without_v_bit_exact(sage, shape):
+    """Variant B's pre-pass (no V): the K statistics then run with two heads
+    per CTA sharing each table load (H_kv even) or one (odd); d = 64 with
+    four heads per quantizer CTA included."""
+    B, H, Hk, N, d = shape
+    w = workloads.get("llm_8p8_b2_h16_n4096_d128").with_(B=B, H=H, H_kv=Hk, N=N, d=d, seed=70 + N)
+    q, k, _ = workloads.generate(w)
+    cos, sin, tcos, tsin = _tables(N, d)
+    tq, tk = to_dev(q, k)
+    scale = 1.0 / np.sqrt(d)
+    got = sage.sage_smooth_quant_qkv_rope(tq, tk, tcos, tsin, None, scale)
+    torch.cuda.synchronize()
+    st, word = sage.sage_get_device_error()
+    assert st == 0, hex(word)
+    qr, kr = oracle.rope(q, cos, sin), oracle.rope(k, cos, sin)
+    eq, edq = oracle.quant_q(qr, scale)
+    ekh, edk, emk = oracle.smooth_quant_k(kr)
+    for n, g, e in zip(("q_hat", "k_hat", "delta_q", "delta_k", "mean_k"), got[:5], (eq, ekh, edq, edk, emk)):
+        g = g.cpu().numpy()
+        if g.dtype == np.float32:
+            assert np.array_equal(_bits(g), _bits(e)), n
+        else:
+            assert np.array_equal(g, e), n
+    assert got[5] is None and got[6] is None
+
+
 def test_rope_prepass_bit_exact_llm_shape(sage):
     w = workloads.get("llm_8p8_b2_h16_n4096_d128")
     q, k, v = workloads.generate(w)
